@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Benchmark: batch-1 INT4 fused-dequant GEMV over a Llama-7B-shaped decode stack.
+
+Workload (one "step" = one decode token through the stack's linear layers):
+  32 layers x {qkv 4096->12288, o 4096->4096, gate 4096->11008, up 4096->11008,
+  down 11008->4096}, INT4 asymmetric RTN, group 128, batch 1, fp16 activations
+  x ~ N(0, 1), weights W = 0.02 * t5 * lognormal_row(0, 0.5) drawn on the GPU
+  with a seeded generator and quantized by qnt_quantize.  160 qnt_gemv calls per
+  step, 3.37 GB of packed weights per step: larger than L2, so every step reads
+  its weights from HBM (no flush needed).
+
+Metric: achieved HBM GB/s from algorithmic bytes (codes + metadata + x + y per
+GEMV) and microseconds per decode layer (step time / 32).  The step's kernels
+are captured once in a CUDA graph and replayed; timing uses CUDA events on the
+launching stream, with a barrier and synchronize around the timed region and
+the max over ranks for N > 1 (each rank runs its own replica: weak scaling).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+LAYERS = 32
+HIDDEN, INTER, QKV = 4096, 11008, 12288
+SHAPES = [("qkv", QKV, HIDDEN), ("o", HIDDEN, HIDDEN), ("gate", INTER, HIDDEN), ("up", INTER, HIDDEN),
+          ("down", HIDDEN, INTER)]   # (name, N, K)
+GROUP = 128
+WORKLOAD = "llama7b_decode_stack_int4_g128_b1"
+METRIC = "4-bit fused-dequant GEMV HBM GB/s (% of peak) and us per decode layer"
+
+
+def algo_bytes_int4(N, K, g=GROUP, M=1):
+    """Algorithmic bytes of one INT4 GEMV: 4-bit codes, fp16 scale + 4-bit zero
+    per group, fp16 x and y."""
+    return N * K // 2 + (N * K // g) * 5 // 2 + 2 * K * M + 2 * N * M
+
+
+STEP_BYTES = LAYERS * sum(algo_bytes_int4(N, K) for _, N, K in SHAPES)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), "measured"
+    return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        win = [s for t, s in self.samples if t0 - 0.15 <= t <= t1 + 0.15]
+        if not win and self.samples:
+            mid = 0.5 * (t0 + t1)
+            win = [min(self.samples, key=lambda ts: abs(ts[0] - mid))[1]]
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        sm = [float(s[1]) for s in win if s[1].replace(".", "").isdigit()]
+        mx = [float(s[2]) for s in win if s[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in win for i in range(4) if len(s) > 5 + i and s[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(win)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def allreduce_max(v, world):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ our arm
+def build_stack(Q, torch, seed_base):
+    """Quantize 32 layers of Llama-7B-shaped weights on the GPU."""
+    from dequant_gemv_rtn_b200 import synth
+    layers = []
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for l in range(LAYERS):
+        mods = []
+        for mi, (name, N, K) in enumerate(SHAPES):
+            d = Q.desc(Q.QNT_INT4_ASYM, N, K, GROUP)
+            W = synth.llama_like_device(N, K, seed=seed_base + 16 * l + mi)
+            codes = torch.empty(Q.qnt_codes_bytes(d), dtype=torch.uint8, device="cuda")
+            meta = torch.empty(Q.qnt_meta_bytes(d), dtype=torch.uint8, device="cuda")
+            Q.qnt_quantize(d, W, codes, meta, st)
+            del W
+            mods.append((name, d, codes, meta))
+        layers.append(mods)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0, f"quantize status {int(st.item())}"
+    return layers
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    from dequant_gemv_rtn_b200 import qnt as Q
+    from dequant_gemv_rtn_b200 import synth
+    torch.cuda.set_device(local)
+    dev_index = torch.cuda.current_device()
+    layers = build_stack(Q, torch, seed_base=1000 * (rank + 1))
+    xs = {K: synth.activations_device(1, K, seed=7 + K, dtype=torch.float16) for K in (HIDDEN, INTER)}
+    ys = {(name, l): torch.empty(N, dtype=torch.float16, device="cuda")
+          for l in range(LAYERS) for name, N, _ in SHAPES}
+    stream = torch.cuda.Stream()
+
+    def step_launches(s):
+        for l, mods in enumerate(layers):
+            for name, d, codes, meta in mods:
+                Q.qnt_gemv(d, codes, meta, xs[d.K], ys[(name, l)], Q.QNT_F16, None, s)
+
+    # eager warm-up (also initializes per-kernel attributes before capture)
+    with torch.cuda.stream(stream):
+        step_launches(stream)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step_launches(torch.cuda.current_stream())
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(dev_index)
+    sampler.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    barrier(world)
+    sampler.stop()
+    ms = e0.elapsed_time(e1)
+    ms = allreduce_max(ms, world)
+    clocks = sampler.summary(t0, t1)
+
+    # per-shape isolated launch times (same kernel, 32 cold layers per graph)
+    per_shape = {}
+    for mi, (name, N, K) in enumerate(SHAPES):
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2, stream=stream):
+            for l in range(LAYERS):
+                _, d, codes, meta = layers[l][mi]
+                Q.qnt_gemv(d, codes, meta, xs[K], ys[(name, l)], Q.QNT_F16, None, torch.cuda.current_stream())
+        for _ in range(3):
+            g2.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 20
+        with torch.cuda.stream(stream):
+            a.record(stream)
+            for _ in range(reps):
+                g2.replay()
+            b.record(stream)
+        torch.cuda.synchronize()
+        us = a.elapsed_time(b) * 1000.0 / (reps * LAYERS)
+        per_shape[f"{name}_{K}x{N}"] = {"us": round(us, 3), "GBps": round(algo_bytes_int4(N, K) / us / 1e3, 1)}
+        del g2
+
+    # end to end through the public API with host buffers: per step, every GEMV's
+    # x goes host->device from pinned memory and every y comes back device->host
+    hx = {K: xs[K].reshape(-1).cpu().pin_memory() for K in (HIDDEN, INTER)}
+    hy = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in ys.items()}
+    dx = {(name, l): torch.empty(K, dtype=torch.float16, device="cuda")
+          for l in range(LAYERS) for name, _, K in SHAPES}
+
+    def e2e_step(s):
+        for l, mods in enumerate(layers):
+            for name, d, codes, meta in mods:
+                xd = dx[(name, l)]
+                xd.copy_(hx[d.K], non_blocking=True)
+                Q.qnt_gemv(d, codes, meta, xd, ys[(name, l)], Q.QNT_F16, None, s)
+                hy[(name, l)].copy_(ys[(name, l)], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        e2e_step(stream)
+    torch.cuda.synchronize()
+    ge = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(ge, stream=stream):
+        e2e_step(torch.cuda.current_stream())
+    for _ in range(max(3, args.warmup)):
+        ge.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, min(args.steps, 200))
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for _ in range(e2e_steps):
+            ge.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = allreduce_max(a.elapsed_time(b), world) / e2e_steps
+    h2d = LAYERS * sum(2 * K for _, _, K in SHAPES)
+    d2h = LAYERS * sum(2 * N for _, N, _ in SHAPES)
+    del ge, graph
+
+    step_ms = ms / args.steps
+    value = world * STEP_BYTES / (step_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peaks()
+    launches = LAYERS * len(SHAPES)
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(step_ms, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int4 weights, fp16 activations, fp32 accumulate", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "layers": LAYERS, "shapes_NxK": [[N, K] for _, N, K in SHAPES],
+                   "group": GROUP, "batch": 1, "bytes_per_step": STEP_BYTES,
+                   "l2": "inputs larger than L2 (3.37 GB of packed weights per step), no flush",
+                   "timing": "CUDA graph of one step replayed; CUDA events on the launching stream",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "us_per_layer": round(step_ms * 1000.0 / LAYERS, 3),
+        "roofline": {"bound": "hbm", "achieved": round(STEP_BYTES / launches / (step_ms * 1e-3 / launches) / 1e9, 1),
+                     "peak": peak, "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy)" if peak_kind == "measured" else "fallback",
+                     "unit": "GB/s", "frac": round(STEP_BYTES / (step_ms * 1e-3) / 1e9 / peak, 4),
+                     "traffic": None, "kernel": "gemv4_kernel<INT4,g128,MB=1>",
+                     "per_launch_bytes": STEP_BYTES // launches},
+        "per_shape_isolated": per_shape,
+        "gpu_launches": launches * args.steps,
+        "clocks": clocks,
+        "e2e": {"value": round(world * STEP_BYTES / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "how": "public C-ABI qnt_gemv per module, x copied from pinned host memory and y copied back "
+                       "for every GEMV, all inside a captured CUDA graph; weights resident"},
+    }
+    return result, layers
+
+
+# ------------------------------------------------------------------ CPU oracle (baseline / reference arm)
+def oracle_layer(torch, seed_base=1000):
+    """One decode layer's weights drawn on the GPU, copied to the host and
+    quantized by the oracle (timed separately from the GEMV)."""
+    from dequant_gemv_rtn_b200 import synth
+    from oracle import oracle as orc
+    mods = []
+    for mi, (name, N, K) in enumerate(SHAPES):
+        W = synth.llama_like_device(N, K, seed=seed_base + mi).cpu().numpy()
+        q = orc.quantize(orc.INT4, W, GROUP)
+        del W
+        x = orc.f2h(synth.activations(1, K, seed=7 + K))
+        mods.append((q, x))
+    return mods
+
+
+def time_oracle_layer(mods, budget_s):
+    from oracle import oracle as orc
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        for q, x in mods:
+            orc.gemm(q, x, 0)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    return (time.perf_counter() - t0) / n, n
+
+
+def cpu_baseline(torch, budget_s=10.0):
+    from oracle import oracle as orc
+    mods = oracle_layer(torch)
+    per_layer_s, n = time_oracle_layer(mods, budget_s)
+    layer_bytes = sum(algo_bytes_int4(N, K) for _, N, K in SHAPES)
+    return {"value": round(layer_bytes / per_layer_s / 1e9, 3), "unit": "GB/s", "cores": orc.threads(),
+            "kind": "oracle",
+            "sample": f"{n} pass(es) of the oracle's binary64 GEMV over one of the 32 decode layers "
+                      f"(5 INT4 g128 matrices, {layer_bytes} algorithmic bytes); {per_layer_s * 1e3:.1f} ms per layer"}
+
+
+def run_reference(args, world, rank, local):
+    import torch
+    if rank != 0:
+        return None
+    torch.cuda.set_device(local)
+    from oracle import oracle as orc
+    mods = oracle_layer(torch)
+    layer_bytes = sum(algo_bytes_int4(N, K) for _, N, K in SHAPES)
+    for _ in range(args.warmup):
+        for q, x in mods:
+            orc.gemm(q, x, 0)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        for q, x in mods:
+            orc.gemm(q, x, 0)
+    per_step = (time.perf_counter() - t0) / args.steps
+    value = layer_bytes / per_step / 1e9
+    sample = (f"each step = the oracle's binary64 GEMV over one decode layer (5 INT4 g128 matrices of the "
+              f"{LAYERS}-layer stack)")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 accumulate",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "layers_per_step": 1, "group": GROUP, "batch": 1},
+            "us_per_layer": round(per_step * 1e6, 1),
+            "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": orc.threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def run_kernel_only(name: str, fmt_name: str, repeats: int = 5):
+    """Small case for profilers: one matrix of the named decode shape, quantized
+    once, then `repeats` qnt_gemv launches (M=1, fp16 x)."""
+    import torch
+    from dequant_gemv_rtn_b200 import qnt as Q
+    from dequant_gemv_rtn_b200 import synth
+    N, K = {n: (N, K) for n, N, K in SHAPES}[name]
+    fmt = Q.FORMATS[fmt_name]
+    d = Q.desc(fmt, N, K, GROUP)
+    W = synth.llama_like_device(N, K, seed=3)
+    codes = torch.empty(Q.qnt_codes_bytes(d), dtype=torch.uint8, device="cuda")
+    meta = torch.empty(max(16, Q.qnt_meta_bytes(d)), dtype=torch.uint8, device="cuda")
+    Q.qnt_quantize(d, W, codes, meta)
+    del W
+    x = synth.activations_device(1, K, seed=5, dtype=torch.float16)
+    y = torch.empty(N, dtype=torch.float16, device="cuda")
+    for _ in range(repeats):
+        Q.qnt_gemv(d, codes, meta, x, y, Q.QNT_F16)
+    torch.cuda.synchronize()
+    print(json.dumps({"kernel_only": name, "fmt": fmt_name, "N": N, "K": K, "launches": repeats,
+                      "y_finite": bool(torch.isfinite(y.float()).all())}))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--kernel-only", choices=[n for n, _, _ in SHAPES], default=None,
+                    help="profiling case: one matrix of this shape, a few GEMV launches")
+    ap.add_argument("--fmt", default="int4", help="format for --kernel-only")
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.kernel_only:
+        run_kernel_only(args.kernel_only, args.fmt)
+        return
+    world, rank, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        r = run_reference(args, world, rank, local)
+        if r is not None:
+            print(json.dumps(r), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    import torch
+    result, _ = run_ours(args, world, rank, local)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(torch, args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

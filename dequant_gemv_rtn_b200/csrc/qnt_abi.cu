@@ -1,0 +1,131 @@
+// qnt_abi.cu -- the C ABI of libqnt: argument validation, buffer sizes and
+// kernel dispatch.  Nothing here allocates memory; every launch goes to the
+// caller's stream.
+#include <cstdint>
+#include <cstring>
+#include <cuda_runtime.h>
+#include "qnt.h"
+
+namespace qnt {
+cudaError_t launch_quantize(const qnt_desc& d, const float* W, void* codes, void* meta, long z0, int* st, cudaStream_t s);
+cudaError_t launch_gemv(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
+                        int M, int xbf16, int* st, cudaStream_t s);
+cudaError_t launch_gemm_tc(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
+                           int M, int xbf16, int* st, cudaStream_t s, bool* handled);
+}  // namespace qnt
+
+namespace {
+
+bool is_4bit(int f) { return f == QNT_INT4_ASYM || f == QNT_FP4_E2M1 || f == QNT_FP4_AFPQ || f == QNT_FP4_RAZER; }
+
+long round_up(long v, long a) { return (v + a - 1) / a * a; }
+
+long n_groups(const qnt_desc& d) { return is_4bit(d.fmt) ? (long)d.N * (d.K / d.group) : (long)d.N; }
+
+// Start of the zero / selector plane inside the metadata buffer.
+long zero_plane(const qnt_desc& d) { return round_up(2 * n_groups(d), 256); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check(const qnt_desc* d) {
+  if (!d) return QNT_ERR_ARG;
+  if (d->fmt < QNT_INT4_ASYM || d->fmt > QNT_FP16) return QNT_ERR_ARG;
+  if (d->N < 1 || d->K < 128 || d->K % 128 != 0) return QNT_ERR_SHAPE;
+  if (d->K > (1 << 20) || d->N > (1 << 24)) return QNT_ERR_SHAPE;
+  if (is_4bit(d->fmt)) {
+    if (d->group != 32 && d->group != 64 && d->group != 128) return QNT_ERR_SHAPE;
+  } else if (d->group != d->K) {
+    return QNT_ERR_SHAPE;
+  }
+  return QNT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qnt_version(void) { return QNT_VERSION; }
+
+int qnt_check_desc(const qnt_desc* desc) { return check(desc); }
+
+size_t qnt_codes_bytes(const qnt_desc* d) {
+  if (check(d) != QNT_OK) return 0;
+  const size_t nk = (size_t)d->N * (size_t)d->K;
+  if (d->fmt == QNT_INT8_PERCHAN) return nk;
+  if (d->fmt == QNT_FP16) return 2 * nk;
+  return nk / 2;
+}
+
+size_t qnt_meta_bytes(const qnt_desc* d) {
+  if (check(d) != QNT_OK) return 0;
+  const long P = n_groups(*d);
+  switch (d->fmt) {
+    case QNT_INT4_ASYM: return (size_t)(zero_plane(*d) + round_up((P + 1) / 2, 4));
+    case QNT_FP4_E2M1: return (size_t)(2 * P);
+    case QNT_FP4_AFPQ: return (size_t)(4 * P);
+    case QNT_FP4_RAZER: return (size_t)(zero_plane(*d) + round_up((P + 3) / 4, 4));
+    case QNT_INT8_PERCHAN: return (size_t)(2 * d->N);
+    default: return 0;
+  }
+}
+
+const char* qnt_strerror(int code) {
+  switch (code) {
+    case QNT_OK: return "ok";
+    case QNT_ERR_ARG: return "invalid argument (null pointer, unknown format or dtype, M out of range)";
+    case QNT_ERR_SHAPE: return "invalid shape (N >= 1, K a positive multiple of 128, group 32/64/128 for 4-bit, K otherwise)";
+    case QNT_ERR_ALIGN: return "buffer not 16-byte aligned";
+    case QNT_ERR_CUDA: return "CUDA launch failed";
+    case QNT_ERR_TIMEOUT: return "device: a bounded wait for an asynchronous copy expired";
+    case QNT_ERR_NONFINITE: return "device: NaN or Inf in the weights";
+    case QNT_ERR_RANGE: return "device: a scale or FP16 code overflowed fp16";
+    default: return "unknown error code";
+  }
+}
+
+int qnt_quantize(const qnt_desc* desc, const float* d_W, void* d_codes, void* d_meta, int* d_status, void* stream) {
+  int e = check(desc);
+  if (e != QNT_OK) return e;
+  if (!d_W || !d_codes || (desc->fmt != QNT_FP16 && !d_meta)) return QNT_ERR_ARG;
+  if (!aligned16(d_W) || !aligned16(d_codes) || (d_meta && !aligned16(d_meta))) return QNT_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long z0 = zero_plane(*desc);
+  if (desc->fmt == QNT_INT4_ASYM || desc->fmt == QNT_FP4_RAZER) {
+    // the zero / selector plane is filled with atomic ORs: clear it first
+    const size_t tail = qnt_meta_bytes(desc) - (size_t)z0;   /* a multiple of 4 bytes */
+    if (cudaMemsetAsync(static_cast<uint8_t*>(d_meta) + z0, 0, tail, s) != cudaSuccess)
+      return QNT_ERR_CUDA;
+  }
+  return qnt::launch_quantize(*desc, d_W, d_codes, d_meta, z0, d_status, s) == cudaSuccess ? QNT_OK : QNT_ERR_CUDA;
+}
+
+int qnt_gemm(const qnt_desc* desc, const void* d_codes, const void* d_meta, const void* d_X, void* d_Y, int M,
+             int xdtype, int* d_status, void* stream) {
+  int e = check(desc);
+  if (e != QNT_OK) return e;
+  if (M < 1 || M > 128) return QNT_ERR_ARG;
+  if (xdtype != QNT_F16 && xdtype != QNT_BF16) return QNT_ERR_ARG;
+  if (!d_codes || !d_X || !d_Y || (desc->fmt != QNT_FP16 && !d_meta)) return QNT_ERR_ARG;
+  if (!aligned16(d_codes) || !aligned16(d_X) || !aligned16(d_Y) || (d_meta && !aligned16(d_meta))) return QNT_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long z0 = zero_plane(*desc);
+  bool handled = false;
+  cudaError_t ce = qnt::launch_gemm_tc(*desc, d_codes, d_meta, z0, d_X, d_Y, M, xdtype == QNT_BF16, d_status, s, &handled);
+  if (!handled) ce = qnt::launch_gemv(*desc, d_codes, d_meta, z0, d_X, d_Y, M, xdtype == QNT_BF16, d_status, s);
+  return ce == cudaSuccess ? QNT_OK : QNT_ERR_CUDA;
+}
+
+int qnt_gemv(const qnt_desc* desc, const void* d_codes, const void* d_meta, const void* d_x, void* d_y, int xdtype,
+             int* d_status, void* stream) {
+  int e = check(desc);
+  if (e != QNT_OK) return e;
+  if (xdtype != QNT_F16 && xdtype != QNT_BF16) return QNT_ERR_ARG;
+  if (!d_codes || !d_x || !d_y || (desc->fmt != QNT_FP16 && !d_meta)) return QNT_ERR_ARG;
+  if (!aligned16(d_codes) || !aligned16(d_x) || !aligned16(d_y) || (d_meta && !aligned16(d_meta))) return QNT_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long z0 = zero_plane(*desc);
+  return qnt::launch_gemv(*desc, d_codes, d_meta, z0, d_x, d_y, 1, xdtype == QNT_BF16, d_status, s) == cudaSuccess
+             ? QNT_OK : QNT_ERR_CUDA;
+}
+
+}  // extern "C"

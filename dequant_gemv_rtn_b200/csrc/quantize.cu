@@ -1,0 +1,299 @@
+// quantize.cu -- RTN group-wise quantization kernels (offline step).
+//
+// Round-to-nearest, data-free ("Is (Selective) Round-To-Nearest Quantization
+// All You Need?", English abstract) with one scale shared per group of g
+// weights ("Revisiting Block-based Quantisation", English abstract) for INT4
+// asymmetric, FP4 E2M1, AFPQ (separate positive / negative scales, "AFPQ"
+// English abstract) and RaZeR (negative-zero code remapped to a per-group
+// special value, "The Power of Negative Zero", method section); plus INT8
+// per-channel and FP16 for selectively raised modules.
+//
+// Bit-exactness: every scalar step is an explicit IEEE binary32 operation
+// (__fdiv_rn, __fsub_rn, rintf, __float2half_rn); RaZeR's squared errors are
+// binary64 (__dmul_rn / __dadd_rn, no contraction) summed as a balanced binary
+// tree in weight order: lane-local pairs, then __shfl_xor with offsets 1, 2, 4...
+#include "common.cuh"
+
+namespace qnt {
+
+// fp16 scale from a binary32 quotient: zero -> 1.0; overflow reported.
+__device__ __forceinline__ uint32_t scale_bits(float q, bool& overflow) {
+  uint32_t h = __half_as_ushort(__float2half_rn(q));
+  if ((h & 0x7FFFu) == 0) h = 0x3C00u;
+  if ((h & 0x7C00u) == 0x7C00u) overflow = true;
+  return h;
+}
+
+// Nearest E2M1 magnitude index of a >= 0: one comparison per midpoint between
+// neighbouring magnitudes {0,.5,1,1.5,2,3,4,6}; at an exact midpoint the index
+// with mantissa bit 0 wins (ties to even), hence '>' vs '>='.
+__device__ __forceinline__ int e2m1_index(float a) {
+  return (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) + (a >= 3.5f) + (a > 5.0f);
+}
+__device__ __forceinline__ double e2m1_mag(int m) {
+  // 0, .5, 1, 1.5, 2, 3, 4, 6 from the bit fields (exponent m>>1, mantissa m&1)
+  int e = m >> 1, f = m & 1;
+  return e == 0 ? 0.5 * f : ldexp(1.0 + 0.5 * f, e - 1);
+}
+__device__ __forceinline__ uint32_t fp4_code(float w, float S) {
+  float v = __fdiv_rn(w, S);
+  int m = e2m1_index(fabsf(v));
+  if (m == 0) return 0;
+  return (v < 0.0f ? 8u : 0u) | (uint32_t)m;
+}
+
+template <int GL>
+__device__ __forceinline__ float group_max(float v) {
+#pragma unroll
+  for (int o = GL / 2; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+template <int GL>
+__device__ __forceinline__ float group_min(float v) {
+#pragma unroll
+  for (int o = GL / 2; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+template <int GL>
+__device__ __forceinline__ double group_tree_sum(double v) {
+#pragma unroll
+  for (int o = 1; o < GL; o <<= 1) v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Position of nibble `e` (0..7, weight within a word) inside the 32-bit word.
+template <int FMT>
+__device__ __forceinline__ int nib_shift(int e) {
+  if (FMT == QNT_INT4_ASYM) return (e & 1) ? 16 + 4 * (e >> 1) : 4 * (e >> 1);  // PI = {0,2,4,6,1,3,5,7}
+  return 4 * e;                                                              // PI = identity
+}
+
+// One warp per (row, 128-weight slot); lane l holds weights 4l..4l+3 of the
+// slot; GL = lanes per group (g / 4).
+template <int FMT, int GL>
+__global__ void __launch_bounds__(256) quantize4_kernel(const float* __restrict__ W, int N, int K,
+                                                        uint8_t* __restrict__ codes, uint8_t* __restrict__ meta,
+                                                        long z0, int* d_status) {
+  const int lane = threadIdx.x & 31;
+  const long warp = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int S = K / kSlot;
+  if (warp >= (long)N * S) return;  // whole warp exits together
+  const long n = warp / S;
+  const int s = (int)(warp % S);
+  const int g = GL * 4;
+  const int G = K / g;
+
+  const float4 w4 = *reinterpret_cast<const float4*>(W + n * K + (long)s * kSlot + 4 * lane);
+  float w[4] = {w4.x, w4.y, w4.z, w4.w};
+  bool bad = !(isfinite(w[0]) && isfinite(w[1]) && isfinite(w[2]) && isfinite(w[3]));
+  bool overflow = false;
+
+  uint32_t c[4];
+  uint32_t m1 = 0, m2 = 0;  // metadata words
+  if (FMT == QNT_INT4_ASYM) {
+    float mn = group_min<GL>(fminf(fminf(w[0], w[1]), fminf(w[2], w[3])));
+    float mx = group_max<GL>(fmaxf(fmaxf(w[0], w[1]), fmaxf(w[2], w[3])));
+    uint32_t sh = scale_bits(__fdiv_rn(__fsub_rn(mx, mn), 15.0f), overflow);
+    float S_ = __half2float(__ushort_as_half((unsigned short)sh));
+    float zf = fminf(fmaxf(rintf(__fdiv_rn(-mn, S_)), 0.0f), 15.0f);
+    int z = (int)zf;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float r = fminf(fmaxf(rintf(__fdiv_rn(w[i], S_)), -64.0f), 64.0f);
+      int q = (int)r + z;
+      c[i] = (uint32_t)min(max(q, 0), 15);
+    }
+    m1 = sh; m2 = (uint32_t)z;
+  } else if (FMT == QNT_FP4_E2M1) {
+    float am = group_max<GL>(fmaxf(fmaxf(fabsf(w[0]), fabsf(w[1])), fmaxf(fabsf(w[2]), fabsf(w[3]))));
+    uint32_t sh = scale_bits(__fdiv_rn(am, 6.0f), overflow);
+    float S_ = __half2float(__ushort_as_half((unsigned short)sh));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) c[i] = fp4_code(w[i], S_);
+    m1 = sh;
+  } else if (FMT == QNT_FP4_AFPQ) {
+    float mn = group_min<GL>(fminf(fminf(w[0], w[1]), fminf(w[2], w[3])));
+    float mx = group_max<GL>(fmaxf(fmaxf(w[0], w[1]), fmaxf(w[2], w[3])));
+    float pos = mx > 0.0f ? mx : 0.0f;
+    float neg = mn < 0.0f ? -mn : 0.0f;
+    uint32_t sp = scale_bits(__fdiv_rn(pos, 6.0f), overflow);
+    uint32_t sn = scale_bits(__fdiv_rn(neg, 6.0f), overflow);
+    float Sp = __half2float(__ushort_as_half((unsigned short)sp));
+    float Sn = __half2float(__ushort_as_half((unsigned short)sn));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) c[i] = w[i] > 0.0f ? fp4_code(w[i], Sp) : (w[i] < 0.0f ? fp4_code(w[i], Sn) : 0u);
+    m1 = sp | (sn << 16);
+  } else {  // RaZeR
+    float am = group_max<GL>(fmaxf(fmaxf(fabsf(w[0]), fabsf(w[1])), fmaxf(fabsf(w[2]), fabsf(w[3]))));
+    double bestE = 0.0;
+    int best = -1;
+    uint32_t best_sh = 0;
+    bool best_ovf = false;
+#pragma unroll 1
+    for (int sel = 0; sel < 4; ++sel) {
+      const double sv = (sel & 2) ? ((sel & 1) ? -8.0 : 8.0) : ((sel & 1) ? -5.0 : 5.0);
+      bool ovf = false;
+      uint32_t sh = scale_bits(__fdiv_rn(am, (sel & 2) ? 8.0f : 6.0f), ovf);
+      float S_ = __half2float(__ushort_as_half((unsigned short)sh));
+      uint32_t cc[4];
+      double sq[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float v = __fdiv_rn(w[i], S_);
+        int m = e2m1_index(fabsf(v));
+        double rv = e2m1_mag(m);
+        uint32_t code = (m == 0) ? 0u : ((v < 0.0f ? 8u : 0u) | (uint32_t)m);
+        if (code & 8u) rv = -rv;
+        double d_reg = fabs((double)v - rv), d_sv = fabs((double)v - sv);
+        if (d_sv < d_reg) { code = 8u; rv = sv; }
+        cc[i] = code;
+        double e = __dadd_rn((double)w[i], -__dmul_rn(rv, (double)S_));
+        sq[i] = __dmul_rn(e, e);
+      }
+      double E = group_tree_sum<GL>(__dadd_rn(__dadd_rn(sq[0], sq[1]), __dadd_rn(sq[2], sq[3])));
+      if (best < 0 || E < bestE) {
+        bestE = E; best = sel; best_sh = sh; best_ovf = ovf;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) c[i] = cc[i];
+      }
+    }
+    overflow = best_ovf;
+    m1 = best_sh; m2 = (uint32_t)best;
+  }
+
+  // status: any non-finite weight in the warp, or a scale overflow
+  if (__any_sync(0xffffffffu, bad)) { if (lane == 0) report(d_status, QNT_ERR_NONFINITE); }
+  else if (overflow && (lane % GL) == 0) report(d_status, QNT_ERR_RANGE);
+
+  // pack: lanes 2m, 2m+1 hold weights 0..3 / 4..7 of word m of the slot
+  const int e0 = (lane & 1) * 4;
+  uint32_t part = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) part |= c[i] << nib_shift<FMT>(e0 + i);
+  uint32_t word = part | __shfl_xor_sync(0xffffffffu, part, 1);
+  if ((lane & 1) == 0) {
+    const int chunk = lane >> 3, j = (lane & 7) >> 1;
+    uint8_t* dst = codes + n * (long)(K / 2) + 16L * ((long)chunk * S + s) + 4 * j;
+    *reinterpret_cast<uint32_t*>(dst) = word;
+  }
+  // metadata: the first lane of each group writes it
+  if ((lane % GL) == 0) {
+    const long f = n * G + (long)s * (kSlot / g) + lane / GL;
+    if (FMT == QNT_FP4_AFPQ) {
+      reinterpret_cast<uint32_t*>(meta)[f] = m1;
+    } else {
+      reinterpret_cast<uint16_t*>(meta)[f] = (uint16_t)m1;
+    }
+    if (FMT == QNT_INT4_ASYM || FMT == QNT_FP4_RAZER) {
+      const int bits = (FMT == QNT_INT4_ASYM) ? 4 : 2;
+      const int per_byte = 8 / bits;
+      const long byte = z0 + f / per_byte;
+      const int shift = (int)(byte & 3) * 8 + bits * (int)(f % per_byte);
+      atomicOr(reinterpret_cast<unsigned int*>(meta + (byte & ~3L)), m2 << shift);
+    }
+  }
+}
+
+// INT8 symmetric per output channel: one block per row.
+__global__ void __launch_bounds__(256) quantize_int8_kernel(const float* __restrict__ W, int K, int8_t* __restrict__ codes,
+                                                            uint16_t* __restrict__ scales, int* d_status) {
+  __shared__ float red[8];
+  __shared__ int badflag;
+  const long n = blockIdx.x;
+  const float* row = W + n * K;
+  if (threadIdx.x == 0) badflag = 0;
+  float am = 0.0f;
+  bool bad = false;
+  for (int k = threadIdx.x * 4; k < K; k += blockDim.x * 4) {
+    float4 v = *reinterpret_cast<const float4*>(row + k);
+    bad |= !(isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w));
+    am = fmaxf(am, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  __syncthreads();
+  if (bad) atomicOr(&badflag, 1);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = am;
+  __syncthreads();
+  am = red[0];
+  for (int i = 1; i < (int)(blockDim.x >> 5); ++i) am = fmaxf(am, red[i]);
+  bool overflow = false;
+  uint32_t sh = scale_bits(__fdiv_rn(am, 127.0f), overflow);
+  float S_ = __half2float(__ushort_as_half((unsigned short)sh));
+  if (threadIdx.x == 0) {
+    scales[n] = (uint16_t)sh;
+    if (badflag) report(d_status, QNT_ERR_NONFINITE);
+    else if (overflow) report(d_status, QNT_ERR_RANGE);
+  }
+  for (int k = threadIdx.x * 4; k < K; k += blockDim.x * 4) {
+    float4 v = *reinterpret_cast<const float4*>(row + k);
+    float f[4] = {v.x, v.y, v.z, v.w};
+    uint32_t packed = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      int q = (int)fminf(fmaxf(rintf(__fdiv_rn(f[i], S_)), -127.0f), 127.0f);
+      packed |= ((uint32_t)q & 0xFFu) << (8 * i);
+    }
+    *reinterpret_cast<uint32_t*>(codes + n * K + k) = packed;
+  }
+}
+
+// FP16: element-wise round to nearest even.
+__global__ void quantize_fp16_kernel(const float* __restrict__ W, long total4, uint16_t* __restrict__ out, int* d_status) {
+  bool bad = false, ovf = false;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total4; i += (long)gridDim.x * blockDim.x) {
+    float4 v = reinterpret_cast<const float4*>(W)[i];
+    float f[4] = {v.x, v.y, v.z, v.w};
+    uint16_t h[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      bad |= !isfinite(f[j]);
+      h[j] = __half_as_ushort(__float2half_rn(f[j]));
+      ovf |= (h[j] & 0x7C00u) == 0x7C00u;
+    }
+    uint2 o;
+    o.x = h[0] | ((uint32_t)h[1] << 16);
+    o.y = h[2] | ((uint32_t)h[3] << 16);
+    reinterpret_cast<uint2*>(out)[i] = o;
+  }
+  if (bad) report(d_status, QNT_ERR_NONFINITE);
+  else if (ovf) report(d_status, QNT_ERR_RANGE);
+}
+
+// ------------------------------------------------------------------ launchers
+template <int FMT>
+static cudaError_t launch_q4(const qnt_desc& d, const float* W, void* codes, void* meta, long z0, int* st, cudaStream_t s) {
+  const long warps = (long)d.N * (d.K / kSlot);
+  const int threads = 256;
+  const long blocks = (warps + 7) / 8;
+  auto* c = static_cast<uint8_t*>(codes);
+  auto* m = static_cast<uint8_t*>(meta);
+  switch (d.group) {
+    case 32: quantize4_kernel<FMT, 8><<<blocks, threads, 0, s>>>(W, d.N, d.K, c, m, z0, st); break;
+    case 64: quantize4_kernel<FMT, 16><<<blocks, threads, 0, s>>>(W, d.N, d.K, c, m, z0, st); break;
+    default: quantize4_kernel<FMT, 32><<<blocks, threads, 0, s>>>(W, d.N, d.K, c, m, z0, st); break;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(const qnt_desc& d, const float* W, void* codes, void* meta, long z0, int* st, cudaStream_t s) {
+  switch (d.fmt) {
+    case QNT_INT4_ASYM: return launch_q4<QNT_INT4_ASYM>(d, W, codes, meta, z0, st, s);
+    case QNT_FP4_E2M1: return launch_q4<QNT_FP4_E2M1>(d, W, codes, meta, z0, st, s);
+    case QNT_FP4_AFPQ: return launch_q4<QNT_FP4_AFPQ>(d, W, codes, meta, z0, st, s);
+    case QNT_FP4_RAZER: return launch_q4<QNT_FP4_RAZER>(d, W, codes, meta, z0, st, s);
+    case QNT_INT8_PERCHAN:
+      quantize_int8_kernel<<<d.N, 256, 0, s>>>(W, d.K, static_cast<int8_t*>(codes), static_cast<uint16_t*>(meta), st);
+      return cudaGetLastError();
+    case QNT_FP16: {
+      const long total4 = (long)d.N * d.K / 4;
+      long blocks = (total4 + 255) / 256;
+      if (blocks > 148 * 16) blocks = 148 * 16;
+      quantize_fp16_kernel<<<blocks, 256, 0, s>>>(W, total4, static_cast<uint16_t*>(codes), st);
+      return cudaGetLastError();
+    }
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace qnt

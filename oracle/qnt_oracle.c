@@ -7,7 +7,7 @@
  * header, table or constant generator with the CUDA library it checks.
  *
  * Sources (the pages give prose, no formulas; the arithmetic below is the
- * plainest reading, each reading tagged [R#] and listed in the design doc):
+ * plainest reading, and each such reading is tagged [R#] below):
  *  - "Is (Selective) Round-To-Nearest Quantization All You Need?" (Kogan,
  *    arXiv 2505.15909), English abstract: data-free RTN weight quantization and
  *    selective higher precision (INT8 / FP16) for chosen modules.
@@ -417,11 +417,13 @@ void o_gemm(int fmt, const uint8_t* codes, const uint16_t* s1, const uint16_t* s
 /*                                                                            */
 /* Metadata (byte offsets within the metadata buffer), G = K/g, P = N*G:      */
 /*   INT4:  fp16 scale[P] at 0; zero nibbles at Z0 = round_up(2P, 256):        */
-/*          group f -> byte Z0 + f/2, low nibble if f even else high nibble.   */
+/*          group f -> byte Z0 + f/2, low nibble if f even else high nibble;   */
+/*          plane length round_up(ceil(P/2), 4) bytes.                         */
 /*   FP4:   fp16 scale[P] at 0.                                                */
 /*   AFPQ:  32-bit word[P] at 0: low half fp16 s+, high half fp16 s-.          */
 /*   RaZeR: fp16 scale[P] at 0; selectors at Z0 = round_up(2P, 256):           */
-/*          group f -> byte Z0 + f/4, bits 2*(f%4)..2*(f%4)+1.                 */
+/*          group f -> byte Z0 + f/4, bits 2*(f%4)..2*(f%4)+1;                 */
+/*          plane length round_up(ceil(P/4), 4) bytes.                         */
 /*   INT8:  fp16 scale[N] at 0.                                                */
 /*   FP16:  no metadata.                                                       */
 /* ------------------------------------------------------------------------- */
@@ -453,10 +455,10 @@ static long round_up(long v, long a) { return (v + a - 1) / a * a; }
 long o_meta_bytes(int fmt, long N, long K, long g) {
   long P = (fmt == OF_INT8 || fmt == OF_FP16) ? N : N * (K / g);
   switch (fmt) {
-    case OF_INT4: return round_up(2 * P, 256) + (P + 1) / 2;
+    case OF_INT4: return round_up(2 * P, 256) + round_up((P + 1) / 2, 4);
     case OF_FP4: return 2 * P;
     case OF_AFPQ: return 4 * P;
-    case OF_RAZER: return round_up(2 * P, 256) + (P + 3) / 4;
+    case OF_RAZER: return round_up(2 * P, 256) + round_up((P + 3) / 4, 4);
     case OF_INT8: return 2 * N;
     default: return 0;
   }

@@ -18,12 +18,12 @@ namespace qnt {
 
 constexpr int kSlot = 128;         // weights per slot (one lane's share of a row)
 constexpr int kChunk = 32;         // weights per 16-byte chunk
-// Every mbarrier wait is a bounded loop of try_wait calls; each call may
-// suspend the thread for up to kSuspendNs (it resumes as soon as the phase
-// completes), so a waiting warp does not steal issue slots, and the total wait
-// is bounded by kMaxTries * kSuspendNs (~2 s) before an error is reported.
-constexpr int kMaxTries = 20000;
-constexpr uint32_t kSuspendNs = 100000;
+// Every mbarrier wait is a bounded loop of try_wait calls, each allowed to
+// suspend the thread for up to kSuspendNs (the thread resumes as soon as the
+// phase completes); the loop gives up after kMaxTries tries (over a second)
+// and the caller reports an error.
+constexpr int kMaxTries = 1 << 20;
+constexpr uint32_t kSuspendNs = 2000;
 
 // ------------------------------------------------------------------ memory
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
@@ -137,6 +137,37 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                :: "r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)) : "memory");
+}
+
+// Same copy with an L2 cache-policy hint (e.g. evict_first for streamed weights).
+__device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t pol) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+               :: "r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(pol) : "memory");
+}
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+// Order this thread's earlier generic-proxy shared-memory accesses before
+// later async-proxy (bulk copy) writes to the same memory.
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t lds_u32(const void* p) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_addr(p)));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds_u16(const void* p) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(smem_addr(p)));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds_u8(const void* p) {
+  unsigned short v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=h"(v) : "r"(smem_addr(p)));
+  return v & 0xFFu;
 }
 
 __device__ __forceinline__ void report(int* d_status, int code) {

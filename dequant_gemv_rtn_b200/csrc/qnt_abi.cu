@@ -60,11 +60,11 @@ size_t qnt_meta_bytes(const qnt_desc* d) {
   if (check(d) != QNT_OK) return 0;
   const long P = n_groups(*d);
   switch (d->fmt) {
-    case QNT_INT4_ASYM: return (size_t)(zero_plane(*d) + round_up((P + 1) / 2, 4));
-    case QNT_FP4_E2M1: return (size_t)(2 * P);
-    case QNT_FP4_AFPQ: return (size_t)(4 * P);
-    case QNT_FP4_RAZER: return (size_t)(zero_plane(*d) + round_up((P + 3) / 4, 4));
-    case QNT_INT8_PERCHAN: return (size_t)(2 * d->N);
+    case QNT_INT4_ASYM: return (size_t)(zero_plane(*d) + round_up((P + 1) / 2, 16));
+    case QNT_FP4_E2M1: return (size_t)round_up(2 * P, 16);
+    case QNT_FP4_AFPQ: return (size_t)round_up(4 * P, 16);
+    case QNT_FP4_RAZER: return (size_t)(zero_plane(*d) + round_up((P + 3) / 4, 16));
+    case QNT_INT8_PERCHAN: return (size_t)round_up(2L * d->N, 16);
     default: return 0;
   }
 }
@@ -92,7 +92,7 @@ int qnt_quantize(const qnt_desc* desc, const float* d_W, void* d_codes, void* d_
   const long z0 = zero_plane(*desc);
   if (desc->fmt == QNT_INT4_ASYM || desc->fmt == QNT_FP4_RAZER) {
     // the zero / selector plane is filled with atomic ORs: clear it first
-    const size_t tail = qnt_meta_bytes(desc) - (size_t)z0;   /* a multiple of 4 bytes */
+    const size_t tail = qnt_meta_bytes(desc) - (size_t)z0;   /* a multiple of 16 bytes */
     if (cudaMemsetAsync(static_cast<uint8_t*>(d_meta) + z0, 0, tail, s) != cudaSuccess)
       return QNT_ERR_CUDA;
   }

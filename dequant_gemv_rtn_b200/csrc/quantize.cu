@@ -173,7 +173,8 @@ __global__ void __launch_bounds__(256) quantize4_kernel(const float* __restrict_
   uint32_t word = part | __shfl_xor_sync(0xffffffffu, part, 1);
   if ((lane & 1) == 0) {
     const int chunk = lane >> 3, j = (lane & 7) >> 1;
-    uint8_t* dst = codes + n * (long)(K / 2) + 16L * ((long)chunk * S + s) + 4 * j;
+    const int tile = s >> 5, L = min(32, S - 32 * tile);   // tile of 32 slots, slots in it
+    uint8_t* dst = codes + n * (long)(K / 2) + 2048L * tile + 16L * (chunk * L + (s & 31)) + 4 * j;
     *reinterpret_cast<uint32_t*>(dst) = word;
   }
   // metadata: the first lane of each group writes it

@@ -112,11 +112,14 @@ typedef struct {
  *
  * 4-bit codes: row n occupies K/2 bytes at byte n*K/2.  The row is split into
  * S = K/128 slots of 128 consecutive weights and each slot into four chunks of
- * 32 weights.  Chunk i (0..3) of slot s is stored as 16 bytes at row offset
- * 16*(i*S + s), so the 32 lanes of a warp that each own one slot read chunk i
- * of 32 consecutive slots with one coalesced 512-byte load.  The 16 bytes are
- * four little-endian 32-bit words; word j holds chunk weights 8j..8j+7 and
- * nibble p (bits 4p..4p+3) of the word holds chunk weight 8j + PI[p]:
+ * 32 weights.  Slots form tiles of 32 (tile t = s/32 holds L = min(32, S-32t)
+ * slots); chunk i (0..3) of slot s is stored as 16 bytes at row offset
+ * 2048*t + 16*(i*L + s%32).  So one tile of a row (4096 weights) is one
+ * contiguous 2 KB run that a single bulk copy fetches, and the 32 lanes of a
+ * warp that each own one slot read chunk i of the tile from 512 contiguous
+ * bytes.  The 16 bytes are four little-endian 32-bit words; word j holds chunk
+ * weights 8j..8j+7 and nibble p (bits 4p..4p+3) of the word holds chunk
+ * weight 8j + PI[p]:
  *   QNT_INT4_ASYM:                 PI = {0,2,4,6,1,3,5,7}
  *   QNT_FP4_E2M1 / AFPQ / RAZER:   PI = {0,1,2,3,4,5,6,7}
  * INT8 codes: row-major int8 [N][K].  FP16 codes: row-major fp16 [N][K].
@@ -124,14 +127,16 @@ typedef struct {
  * Metadata buffer (byte offsets), G = K/group, P = N*G, group f = n*G + j:
  *   INT4:  fp16 scale[P] at 0; 4-bit zeros from Z0 = round_up(2P, 256):
  *          zero of group f in byte Z0 + f/2, low nibble when f is even;
- *          the zero plane is round_up(ceil(P/2), 4) bytes long.
+ *          the zero plane is round_up(ceil(P/2), 16) bytes long.
  *   FP4:   fp16 scale[P] at 0.
  *   AFPQ:  32-bit word[P] at 0: bits 0..15 = fp16 s+, bits 16..31 = fp16 s-.
  *   RaZeR: fp16 scale[P] at 0; 2-bit selectors from Z0 = round_up(2P, 256):
  *          selector of group f in byte Z0 + f/4, bits 2*(f%4)..2*(f%4)+1;
- *          the selector plane is round_up(ceil(P/4), 4) bytes long.
+ *          the selector plane is round_up(ceil(P/4), 16) bytes long.
  *   INT8:  fp16 scale[N] at 0.
  *   FP16:  none (qnt_meta_bytes returns 0).
+ * Every metadata length is rounded up to a multiple of 16 bytes (the GEMV
+ * kernels stage whole 16-byte-aligned metadata ranges with bulk copies).
  */
 
 /* Bytes of packed codes / metadata for a descriptor; 0 if it is invalid. */

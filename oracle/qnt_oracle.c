@@ -407,8 +407,10 @@ void o_gemm(int fmt, const uint8_t* codes, const uint16_t* s1, const uint16_t* s
 /*                                                                            */
 /* 4-bit formats: row n occupies K/2 bytes starting at n*K/2.  The row is     */
 /* split into S = K/128 slots of 128 consecutive weights; each slot into four */
-/* chunks of 32 weights.  Chunk i (0..3) of slot s is stored as 16 bytes at   */
-/* row offset 16*(i*S + s).  Those 16 bytes are four little-endian 32-bit     */
+/* chunks of 32 weights.  Slots are grouped in tiles of 32 (tile t = s/32,    */
+/* L = min(32, S - 32t) slots in the tile); chunk i (0..3) of slot s is       */
+/* stored as 16 bytes at row offset 2048*t + 16*(i*L + s%32).  Those 16 bytes */
+/* are four little-endian 32-bit                                              */
 /* words; word j holds chunk weights 8j..8j+7; nibble p (bits 4p..4p+3) of    */
 /* the word holds chunk weight 8j + PI[p], with                               */
 /*   INT4:            PI = {0,2,4,6,1,3,5,7}                                   */
@@ -418,12 +420,13 @@ void o_gemm(int fmt, const uint8_t* codes, const uint16_t* s1, const uint16_t* s
 /* Metadata (byte offsets within the metadata buffer), G = K/g, P = N*G:      */
 /*   INT4:  fp16 scale[P] at 0; zero nibbles at Z0 = round_up(2P, 256):        */
 /*          group f -> byte Z0 + f/2, low nibble if f even else high nibble;   */
-/*          plane length round_up(ceil(P/2), 4) bytes.                         */
+/*          plane length round_up(ceil(P/2), 16) bytes.                        */
 /*   FP4:   fp16 scale[P] at 0.                                                */
 /*   AFPQ:  32-bit word[P] at 0: low half fp16 s+, high half fp16 s-.          */
 /*   RaZeR: fp16 scale[P] at 0; selectors at Z0 = round_up(2P, 256):           */
 /*          group f -> byte Z0 + f/4, bits 2*(f%4)..2*(f%4)+1;                 */
-/*          plane length round_up(ceil(P/4), 4) bytes.                         */
+/*          plane length round_up(ceil(P/4), 16) bytes.                        */
+/*   Every metadata buffer length is a multiple of 16 bytes.                  */
 /*   INT8:  fp16 scale[N] at 0.                                                */
 /*   FP16:  no metadata.                                                       */
 /* ------------------------------------------------------------------------- */
@@ -437,10 +440,11 @@ static void nib_pos(int fmt, long n, long k, int K, long* byte, int* hi) {
   const int* pi = (fmt == OF_INT4) ? PI_INT4 : PI_FP4;
   long S = K / 128;
   long s = k / 128, i = (k % 128) / 32, c = k % 32;   /* slot, chunk, weight in chunk */
+  long t = s / 32, L = (S - 32 * t) < 32 ? (S - 32 * t) : 32;   /* tile, slots in tile */
   long j = c / 8, e = c % 8;                            /* word, weight in word */
   int p = 0;
-  for (int t = 0; t < 8; t++) if (pi[t] == e) p = t;   /* nibble holding weight e */
-  *byte = n * (long)(K / 2) + 16 * (i * S + s) + 4 * j + p / 2;
+  for (int q = 0; q < 8; q++) if (pi[q] == e) p = q;   /* nibble holding weight e */
+  *byte = n * (long)(K / 2) + 2048 * t + 16 * (i * L + s % 32) + 4 * j + p / 2;
   *hi = p & 1;
 }
 
@@ -455,11 +459,11 @@ static long round_up(long v, long a) { return (v + a - 1) / a * a; }
 long o_meta_bytes(int fmt, long N, long K, long g) {
   long P = (fmt == OF_INT8 || fmt == OF_FP16) ? N : N * (K / g);
   switch (fmt) {
-    case OF_INT4: return round_up(2 * P, 256) + round_up((P + 1) / 2, 4);
-    case OF_FP4: return 2 * P;
-    case OF_AFPQ: return 4 * P;
-    case OF_RAZER: return round_up(2 * P, 256) + round_up((P + 3) / 4, 4);
-    case OF_INT8: return 2 * N;
+    case OF_INT4: return round_up(2 * P, 256) + round_up((P + 1) / 2, 16);
+    case OF_FP4: return round_up(2 * P, 16);
+    case OF_AFPQ: return round_up(4 * P, 16);
+    case OF_RAZER: return round_up(2 * P, 256) + round_up((P + 3) / 4, 16);
+    case OF_INT8: return round_up(2 * N, 16);
     default: return 0;
   }
 }

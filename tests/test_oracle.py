@@ -437,16 +437,27 @@ def test_pack_unpack_roundtrip(orc, fmt):
 
 def test_layout_hand_positions(orc):
     """A few byte/nibble positions worked out by hand from the layout text."""
-    N, K, g = 2, 256, 128                      # S = 2 slots per row, 128 bytes per row
+    N, K, g = 2, 256, 128                      # S = 2 slots (one tile, L = 2), 128 bytes per row
     for fmt, pi in [(orc.INT4, [0, 2, 4, 6, 1, 3, 5, 7]), (orc.FP4, list(range(8)))]:
         codes = np.zeros((N, K), np.uint8)
         # weight (n=1, k=128+32*2+8*1+pi[5]) -> slot 1, chunk 2, word 1, nibble 5:
-        # byte = 1*128 + 16*(2*2+1) + 4*1 + 2 = 214, high nibble
+        # byte = 1*128 + 2048*0 + 16*(2*2+1) + 4*1 + 2 = 214, high nibble
         k = 128 + 64 + 8 + pi[5]
         codes[1, k] = 0xB
         q = orc.Quant(fmt, N, K, g, codes, np.zeros(4, np.uint16), np.zeros(4, np.uint16), np.zeros(4, np.uint8))
         pc, _ = orc.pack(q)
         assert pc[214] == 0xB0 and pc.sum() == 0xB0
+    # second tile of a K = 4224 row (S = 33: tile 1 holds L = 1 slot):
+    # weight (n=0, k=32*128 + 32*3 + 8*2 + pi[6]) -> slot 32, chunk 3, word 2, nibble 6
+    # byte = 2048*1 + 16*(3*1 + 0) + 4*2 + 3 = 2107, low nibble
+    K2 = 4224
+    for fmt, pi in [(orc.INT4, [0, 2, 4, 6, 1, 3, 5, 7]), (orc.FP4, list(range(8)))]:
+        codes = np.zeros((1, K2), np.uint8)
+        codes[0, 4096 + 96 + 16 + pi[6]] = 0x5
+        G2 = K2 // 128
+        q = orc.Quant(fmt, 1, K2, 128, codes, np.zeros(G2, np.uint16), np.zeros(G2, np.uint16), np.zeros(G2, np.uint8))
+        pc, _ = orc.pack(q)
+        assert pc[2107] == 0x05 and pc.sum() == 5
         # weight (n=0, k=pi[0]) -> byte 0, low nibble
         codes[:] = 0
         codes[0, pi[0]] = 0x7

@@ -1,0 +1,31 @@
+// kernels.h -- host-side entry points of the libqnt kernels (internal; the C
+// ABI in qnt_abi.cu validates arguments and dispatches to these).
+#pragma once
+#include <cuda_runtime.h>
+#include "qnt.h"
+
+namespace qnt {
+
+// Streaming multiprocessors of the current device (cached per device).
+int num_sms();
+// Dynamic shared memory that one CTA may request on sm_100.
+constexpr int kMaxDynSmem = 227 * 1024;
+// Raise a kernel's dynamic shared-memory limit once per process and device;
+// later launches make no attribute calls, so they are safe inside stream capture.
+cudaError_t configure_smem(const void* fn);
+
+// RTN quantization (quantize.cu).
+cudaError_t launch_quantize(const qnt_desc& d, const float* W, void* codes, void* meta, long z0, int* st,
+                            cudaStream_t s);
+
+// Y[m] = W x[m] for m < M on CUDA cores, any format (gemv.cu).
+cudaError_t launch_gemv_simt(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X,
+                             void* Y, int M, int xbf16, int* st, cudaStream_t s);
+
+// Y[m] = W x[m] for m < M on the tensor cores (gemv_tc.cu).  Returns with
+// *handled = false, launching nothing, when the tensor-core kernel does not
+// take this format / batch / shape.
+cudaError_t launch_gemv_tc(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
+                           int M, int xbf16, int* st, cudaStream_t s, bool* handled);
+
+}  // namespace qnt

@@ -6,13 +6,8 @@
 #include <cuda_runtime.h>
 #include "qnt.h"
 
-namespace qnt {
-cudaError_t launch_quantize(const qnt_desc& d, const float* W, void* codes, void* meta, long z0, int* st, cudaStream_t s);
-cudaError_t launch_gemv(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
-                        int M, int xbf16, int* st, cudaStream_t s);
-cudaError_t launch_gemm_tc(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
-                           int M, int xbf16, int* st, cudaStream_t s, bool* handled);
-}  // namespace qnt
+#include <cstdlib>
+#include "kernels.h"
 
 namespace {
 
@@ -40,6 +35,24 @@ int check(const qnt_desc* d) {
   return QNT_OK;
 }
 
+// Y[m] = W x[m], m < M: the tensor-core kernel where it applies, else the
+// CUDA-core kernel.  QNT_FORCE_SIMT=1 in the environment selects the CUDA-core
+// kernel everywhere (used to test both paths on the same inputs).
+cudaError_t dispatch_gemm(const qnt_desc& d, const void* codes, const void* meta, const void* X, void* Y, int M,
+                          int xbf16, int* st, cudaStream_t s) {
+  static const bool force_simt = [] {
+    const char* v = std::getenv("QNT_FORCE_SIMT");
+    return v && v[0] == '1';
+  }();
+  const long z0 = zero_plane(d);
+  if (!force_simt) {
+    bool handled = false;
+    cudaError_t e = qnt::launch_gemv_tc(d, codes, meta, z0, X, Y, M, xbf16, st, s, &handled);
+    if (handled || e != cudaSuccess) return e;
+  }
+  return qnt::launch_gemv_simt(d, codes, meta, z0, X, Y, M, xbf16, st, s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -53,7 +66,7 @@ size_t qnt_codes_bytes(const qnt_desc* d) {
   const size_t nk = (size_t)d->N * (size_t)d->K;
   if (d->fmt == QNT_INT8_PERCHAN) return nk;
   if (d->fmt == QNT_FP16) return 2 * nk;
-  return nk / 2;
+  return ((size_t)d->N + 7) / 8 * 8 * (size_t)d->K / 2;   // 4-bit: whole row groups of eight
 }
 
 size_t qnt_meta_bytes(const qnt_desc* d) {
@@ -108,11 +121,8 @@ int qnt_gemm(const qnt_desc* desc, const void* d_codes, const void* d_meta, cons
   if (!d_codes || !d_X || !d_Y || (desc->fmt != QNT_FP16 && !d_meta)) return QNT_ERR_ARG;
   if (!aligned16(d_codes) || !aligned16(d_X) || !aligned16(d_Y) || (d_meta && !aligned16(d_meta))) return QNT_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const long z0 = zero_plane(*desc);
-  bool handled = false;
-  cudaError_t ce = qnt::launch_gemm_tc(*desc, d_codes, d_meta, z0, d_X, d_Y, M, xdtype == QNT_BF16, d_status, s, &handled);
-  if (!handled) ce = qnt::launch_gemv(*desc, d_codes, d_meta, z0, d_X, d_Y, M, xdtype == QNT_BF16, d_status, s);
-  return ce == cudaSuccess ? QNT_OK : QNT_ERR_CUDA;
+  return dispatch_gemm(*desc, d_codes, d_meta, d_X, d_Y, M, xdtype == QNT_BF16, d_status, s) == cudaSuccess
+             ? QNT_OK : QNT_ERR_CUDA;
 }
 
 int qnt_gemv(const qnt_desc* desc, const void* d_codes, const void* d_meta, const void* d_x, void* d_y, int xdtype,
@@ -123,8 +133,7 @@ int qnt_gemv(const qnt_desc* desc, const void* d_codes, const void* d_meta, cons
   if (!d_codes || !d_x || !d_y || (desc->fmt != QNT_FP16 && !d_meta)) return QNT_ERR_ARG;
   if (!aligned16(d_codes) || !aligned16(d_x) || !aligned16(d_y) || (d_meta && !aligned16(d_meta))) return QNT_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const long z0 = zero_plane(*desc);
-  return qnt::launch_gemv(*desc, d_codes, d_meta, z0, d_x, d_y, 1, xdtype == QNT_BF16, d_status, s) == cudaSuccess
+  return dispatch_gemm(*desc, d_codes, d_meta, d_x, d_y, 1, xdtype == QNT_BF16, d_status, s) == cudaSuccess
              ? QNT_OK : QNT_ERR_CUDA;
 }
 

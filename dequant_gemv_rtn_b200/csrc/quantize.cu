@@ -13,6 +13,7 @@
 // binary64 (__dmul_rn / __dadd_rn, no contraction) summed as a balanced binary
 // tree in weight order: lane-local pairs, then __shfl_xor with offsets 1, 2, 4...
 #include "common.cuh"
+#include "kernels.h"
 
 namespace qnt {
 
@@ -59,13 +60,6 @@ __device__ __forceinline__ double group_tree_sum(double v) {
 #pragma unroll
   for (int o = 1; o < GL; o <<= 1) v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
-}
-
-// Position of nibble `e` (0..7, weight within a word) inside the 32-bit word.
-template <int FMT>
-__device__ __forceinline__ int nib_shift(int e) {
-  if (FMT == QNT_INT4_ASYM) return (e & 1) ? 16 + 4 * (e >> 1) : 4 * (e >> 1);  // PI = {0,2,4,6,1,3,5,7}
-  return 4 * e;                                                              // PI = identity
 }
 
 // One warp per (row, 128-weight slot); lane l holds weights 4l..4l+3 of the
@@ -165,16 +159,28 @@ __global__ void __launch_bounds__(256) quantize4_kernel(const float* __restrict_
   if (__any_sync(0xffffffffu, bad)) { if (lane == 0) report(d_status, QNT_ERR_NONFINITE); }
   else if (overflow && (lane % GL) == 0) report(d_status, QNT_ERR_RANGE);
 
-  // pack: lanes 2m, 2m+1 hold weights 0..3 / 4..7 of word m of the slot
-  const int e0 = (lane & 1) * 4;
+  // pack: the 8 lanes of a 32-weight chunk (lanes 8c..8c+7, chunk weights
+  // 4(l%8)..4(l%8)+3) build its four words, laid out as the header describes
   uint32_t part = 0;
+  int partner, j;
+  bool writer;
+  if (FMT == QNT_INT4_ASYM) {
+    // chunk weight e = 4(l%8)+i sits in word (l%4), nibble h + 2(i/2) + 4(i%2) with h = (l%8)/4
+    const int h = (lane >> 2) & 1;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) part |= c[i] << nib_shift<FMT>(e0 + i);
-  uint32_t word = part | __shfl_xor_sync(0xffffffffu, part, 1);
-  if ((lane & 1) == 0) {
-    const int chunk = lane >> 3, j = (lane & 7) >> 1;
-    const int tile = s >> 5, L = min(32, S - 32 * tile);   // tile of 32 slots, slots in it
-    uint8_t* dst = codes + n * (long)(K / 2) + 2048L * tile + 16L * (chunk * L + (s & 31)) + 4 * j;
+    for (int i = 0; i < 4; ++i) part |= c[i] << (4 * (h + 2 * (i >> 1) + 4 * (i & 1)));
+    partner = 4; j = lane & 3; writer = h == 0;
+  } else {
+    // chunk weight e = 4(l%8)+i sits in word e/8, nibble e%8
+#pragma unroll
+    for (int i = 0; i < 4; ++i) part |= c[i] << (4 * (4 * (lane & 1) + i));
+    partner = 1; j = (lane & 7) >> 1; writer = (lane & 1) == 0;
+  }
+  const uint32_t word = part | __shfl_xor_sync(0xffffffffu, part, partner);
+  if (writer) {
+    // row group n/8 (4K bytes), block s (512 bytes), row n%8 (64 bytes), swizzled chunk
+    const int i8 = (int)(n & 7), c = lane >> 3;
+    uint8_t* dst = codes + (n >> 3) * 4L * K + 512L * s + 64 * i8 + 16 * (c ^ ((i8 >> 1) & 3)) + 4 * j;
     *reinterpret_cast<uint32_t*>(dst) = word;
   }
   // metadata: the first lane of each group writes it

@@ -110,18 +110,22 @@ typedef struct {
 /*
  * Packed storage layout (one layout serves qnt_gemv and qnt_gemm).
  *
- * 4-bit codes: row n occupies K/2 bytes at byte n*K/2.  The row is split into
- * S = K/128 slots of 128 consecutive weights and each slot into four chunks of
- * 32 weights.  Slots form tiles of 32 (tile t = s/32 holds L = min(32, S-32t)
- * slots); chunk i (0..3) of slot s is stored as 16 bytes at row offset
- * 2048*t + 16*(i*L + s%32).  So one tile of a row (4096 weights) is one
- * contiguous 2 KB run that a single bulk copy fetches, and the 32 lanes of a
- * warp that each own one slot read chunk i of the tile from 512 contiguous
- * bytes.  The 16 bytes are four little-endian 32-bit words; word j holds chunk
- * weights 8j..8j+7 and nibble p (bits 4p..4p+3) of the word holds chunk
- * weight 8j + PI[p]:
- *   QNT_INT4_ASYM:                 PI = {0,2,4,6,1,3,5,7}
- *   QNT_FP4_E2M1 / AFPQ / RAZER:   PI = {0,1,2,3,4,5,6,7}
+ * 4-bit codes: rows are stored in groups of eight.  Row group R = n/8 occupies
+ * 4K bytes at byte R*4K (the buffer holds ceil(N/8)*8 rows; the contents of
+ * padding rows are unspecified and never reach a result).  Within a group,
+ * block b (weights 128b..128b+127 of each of its eight rows) occupies 512
+ * bytes at offset 512b; row i = n%8 sits at offset 64i inside the block as four
+ * 16-byte chunks, chunk c (weights 128b+32c .. 128b+32c+31 of the row) at byte
+ * 64i + 16*(c XOR ((i/2) % 4)).  The 16 bytes of a chunk are four little-endian
+ * 32-bit words, and nibble p (bits 4p..4p+3) of word j holds chunk weight
+ *   QNT_INT4_ASYM:                 16*(p%2) + 4j + 2*((p/2)%2) + p/4
+ *   QNT_FP4_E2M1 / AFPQ / RAZER:   8j + p
+ * So 256 consecutive weights of eight rows are one contiguous 1 KB run (one
+ * bulk copy), eight threads that read the same chunk of eight rows of a group
+ * hit distinct shared-memory bank groups, and the INT4 order turns a word into
+ * fp16 pairs with two masks and one shift (low nibbles give chunk weights 0..15
+ * in order, high nibbles 16..31).  FP4-family bytes hold two consecutive
+ * weights, low nibble first.
  * INT8 codes: row-major int8 [N][K].  FP16 codes: row-major fp16 [N][K].
  *
  * Metadata buffer (byte offsets), G = K/group, P = N*G, group f = n*G + j:

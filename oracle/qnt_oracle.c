@@ -405,16 +405,17 @@ void o_gemm(int fmt, const uint8_t* codes, const uint16_t* s1, const uint16_t* s
 /* Packed layout (the library's documented storage format, restated from its */
 /* text; this is the independent unpacker/packer used by the tests).           */
 /*                                                                            */
-/* 4-bit formats: row n occupies K/2 bytes starting at n*K/2.  The row is     */
-/* split into S = K/128 slots of 128 consecutive weights; each slot into four */
-/* chunks of 32 weights.  Slots are grouped in tiles of 32 (tile t = s/32,    */
-/* L = min(32, S - 32t) slots in the tile); chunk i (0..3) of slot s is       */
-/* stored as 16 bytes at row offset 2048*t + 16*(i*L + s%32).  Those 16 bytes */
-/* are four little-endian 32-bit                                              */
-/* words; word j holds chunk weights 8j..8j+7; nibble p (bits 4p..4p+3) of    */
-/* the word holds chunk weight 8j + PI[p], with                               */
-/*   INT4:            PI = {0,2,4,6,1,3,5,7}                                   */
-/*   FP4, AFPQ, RaZeR: PI = {0,1,2,3,4,5,6,7}                                  */
+/* 4-bit formats: rows are stored in groups of eight (row group R = n/8; the  */
+/* codes buffer holds ceil(N/8)*8 rows, padding rows unspecified).  Row group */
+/* R occupies 4K bytes starting at R*4K.  Within it, block b (weights         */
+/* 128b..128b+127 of each of the eight rows) occupies 512 bytes at 512b; row  */
+/* i = n%8 of the group sits at 64i inside the block as four 16-byte chunks,  */
+/* and chunk c (weights 128b+32c..128b+32c+31 of the row) is stored at chunk  */
+/* position c XOR ((i/2) % 4), i.e. at byte 64i + 16*(c ^ ((i/2) % 4)).       */
+/* The 16 bytes of a chunk are four little-endian 32-bit words; nibble p      */
+/* (bits 4p..4p+3) of word j holds chunk weight                               */
+/*   INT4:             16*(p%2) + 4j + 2*((p/2)%2) + p/4                      */
+/*   FP4, AFPQ, RaZeR: 8j + p                                                 */
 /* INT8: codes row-major, one signed byte per weight.  FP16: row-major fp16.  */
 /*                                                                            */
 /* Metadata (byte offsets within the metadata buffer), G = K/g, P = N*G:      */
@@ -431,27 +432,30 @@ void o_gemm(int fmt, const uint8_t* codes, const uint16_t* s1, const uint16_t* s
 /*   FP16:  no metadata.                                                       */
 /* ------------------------------------------------------------------------- */
 
-static const int PI_INT4[8] = {0, 2, 4, 6, 1, 3, 5, 7};
-static const int PI_FP4[8] = {0, 1, 2, 3, 4, 5, 6, 7};
-
 /* Byte offset within the packed codes and nibble index (0 low, 1 high) of
- * weight (n, k) for a 4-bit format. */
+ * weight (n, k) for a 4-bit format: invert the chunk-weight formula above. */
 static void nib_pos(int fmt, long n, long k, int K, long* byte, int* hi) {
-  const int* pi = (fmt == OF_INT4) ? PI_INT4 : PI_FP4;
-  long S = K / 128;
-  long s = k / 128, i = (k % 128) / 32, c = k % 32;   /* slot, chunk, weight in chunk */
-  long t = s / 32, L = (S - 32 * t) < 32 ? (S - 32 * t) : 32;   /* tile, slots in tile */
-  long j = c / 8, e = c % 8;                            /* word, weight in word */
-  int p = 0;
-  for (int q = 0; q < 8; q++) if (pi[q] == e) p = q;   /* nibble holding weight e */
-  *byte = n * (long)(K / 2) + 2048 * t + 16 * (i * L + s % 32) + 4 * j + p / 2;
+  long R = n / 8, i = n % 8;            /* row group, row within the group */
+  long b = k / 128, c = (k % 128) / 32; /* block, chunk within the row's block */
+  long e = k % 32;                      /* weight within the chunk */
+  long j;
+  int p;
+  if (fmt == OF_INT4) {
+    long h = e / 16, r = e % 16;        /* h = p%2; r = 4j + 2*((p/2)%2) + p/4 */
+    j = r / 4;
+    p = (int)(h + 2 * ((r % 4) / 2) + 4 * (r % 2));
+  } else {
+    j = e / 8;
+    p = (int)(e % 8);
+  }
+  *byte = R * 4L * K + 512 * b + 64 * i + 16 * (c ^ ((i / 2) % 4)) + 4 * j + p / 2;
   *hi = p & 1;
 }
 
 long o_codes_bytes(int fmt, long N, long K) {
   if (fmt == OF_INT8) return N * K;
   if (fmt == OF_FP16) return 2 * N * K;
-  return N * K / 2;
+  return (N + 7) / 8 * 8 * K / 2;   /* 4-bit: whole row groups of eight */
 }
 
 static long round_up(long v, long a) { return (v + a - 1) / a * a; }

@@ -437,30 +437,51 @@ def test_pack_unpack_roundtrip(orc, fmt):
 
 def test_layout_hand_positions(orc):
     """A few byte/nibble positions worked out by hand from the layout text."""
-    N, K, g = 2, 256, 128                      # S = 2 slots (one tile, L = 2), 128 bytes per row
-    for fmt, pi in [(orc.INT4, [0, 2, 4, 6, 1, 3, 5, 7]), (orc.FP4, list(range(8)))]:
+    N, K, g = 2, 256, 128                      # one row group of 8 rows, 4K = 1024 bytes
+    # INT4, weight (n=1, k=187): row group 0, row i=1, block 1, chunk c=1, chunk weight 27:
+    # p%2 = 1, r = 11 -> word 2, (p/2)%2 = 1, p/4 = 1 -> p = 7;
+    # byte = 512*1 + 64*1 + 16*(1 ^ 0) + 4*2 + 3 = 603, high nibble.
+    # FP4, weight (n=1, k=183): block 1, chunk 1, chunk weight 23 -> word 2, p = 7 -> byte 603.
+    for fmt, k in [(orc.INT4, 187), (orc.FP4, 183)]:
         codes = np.zeros((N, K), np.uint8)
-        # weight (n=1, k=128+32*2+8*1+pi[5]) -> slot 1, chunk 2, word 1, nibble 5:
-        # byte = 1*128 + 2048*0 + 16*(2*2+1) + 4*1 + 2 = 214, high nibble
-        k = 128 + 64 + 8 + pi[5]
         codes[1, k] = 0xB
         q = orc.Quant(fmt, N, K, g, codes, np.zeros(4, np.uint16), np.zeros(4, np.uint16), np.zeros(4, np.uint8))
         pc, _ = orc.pack(q)
-        assert pc[214] == 0xB0 and pc.sum() == 0xB0
-    # second tile of a K = 4224 row (S = 33: tile 1 holds L = 1 slot):
-    # weight (n=0, k=32*128 + 32*3 + 8*2 + pi[6]) -> slot 32, chunk 3, word 2, nibble 6
-    # byte = 2048*1 + 16*(3*1 + 0) + 4*2 + 3 = 2107, low nibble
+        assert pc.size == 1024
+        assert pc[603] == 0xB0 and pc.sum() == 0xB0
+    # INT4 low-nibble half, row 0, chunk 2: k = 76..79 -> word 3, p = 0, 4, 2, 6 -> bytes 44, 46, 45, 47
+    for k, byte in [(64 + 12 + 1, 46), (64 + 12 + 2, 45), (64 + 12 + 3, 47), (64 + 12, 44)]:
+        codes = np.zeros((N, K), np.uint8)
+        codes[0, k] = 0x6
+        q = orc.Quant(orc.INT4, N, K, g, codes, np.zeros(4, np.uint16), np.zeros(4, np.uint16), np.zeros(4, np.uint8))
+        pc, _ = orc.pack(q)
+        assert pc[byte] == 0x06 and pc.sum() == 6, (k, byte)
+    # chunk swizzle in the second row group: n = 13 -> group 1, row i = 5, (i/2)%4 = 2;
+    # k = 44 -> block 0, chunk 1 -> chunk position 1 ^ 2 = 3;
+    # FP4: chunk weight 12 -> word 1, p = 4 -> byte 1024 + 64*5 + 16*3 + 4 + 2 = 1398, low nibble
+    # INT4: chunk weight 12 -> p%2 = 0, r = 12 -> word 3, p = 0 -> byte 1024 + 320 + 48 + 12 = 1404, low
+    N2 = 14
+    for fmt, byte in [(orc.FP4, 1398), (orc.INT4, 1404)]:
+        codes = np.zeros((N2, K), np.uint8)
+        codes[13, 44] = 0x9
+        G2 = N2 * 2
+        q = orc.Quant(fmt, N2, K, g, codes, np.zeros(G2, np.uint16), np.zeros(G2, np.uint16), np.zeros(G2, np.uint8))
+        pc, _ = orc.pack(q)
+        assert pc.size == 16 * 128
+        assert pc[byte] == 0x09 and pc.sum() == 9
+    # last weight of a K = 4224 row (33 blocks): k = 4223 -> block 32, chunk 3, chunk weight 31;
+    # INT4 and FP4 both put it in word 3, p = 7 -> byte 512*32 + 16*3 + 12 + 3 = 16447, high nibble
     K2 = 4224
-    for fmt, pi in [(orc.INT4, [0, 2, 4, 6, 1, 3, 5, 7]), (orc.FP4, list(range(8)))]:
+    G2 = K2 // 128
+    for fmt in (orc.INT4, orc.FP4):
         codes = np.zeros((1, K2), np.uint8)
-        codes[0, 4096 + 96 + 16 + pi[6]] = 0x5
-        G2 = K2 // 128
+        codes[0, K2 - 1] = 0x5
         q = orc.Quant(fmt, 1, K2, 128, codes, np.zeros(G2, np.uint16), np.zeros(G2, np.uint16), np.zeros(G2, np.uint8))
         pc, _ = orc.pack(q)
-        assert pc[2107] == 0x05 and pc.sum() == 5
-        # weight (n=0, k=pi[0]) -> byte 0, low nibble
+        assert pc.size == 8 * K2 // 2
+        assert pc[16447] == 0x50 and pc.sum() == 0x50
         codes[:] = 0
-        codes[0, pi[0]] = 0x7
+        codes[0, 0] = 0x7                       # weight 0 -> byte 0, low nibble (both formats)
         pc, _ = orc.pack(q)
         assert pc[0] == 0x07 and pc.sum() == 7
     # metadata: INT4 zero of group f=3 -> byte round_up(2*4, 256) + 1, high nibble

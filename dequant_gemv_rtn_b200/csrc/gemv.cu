@@ -118,6 +118,62 @@ __device__ __forceinline__ GroupMeta group_meta(const uint8_t* meta, long z0, lo
   return g;
 }
 
+// The metadata of a CTA's rows, staged in shared memory: 16-byte-aligned
+// supersets of the scale plane (A bytes per group) and of the zero / selector
+// plane (B bits per group) that the rows [r_lo, r_hi) use.
+template <int FMT> struct MetaPlanes {
+  static constexpr int A = (FMT == QNT_FP4_AFPQ) ? 4 : 2;
+  static constexpr int B = (FMT == QNT_INT4_ASYM) ? 4 : (FMT == QNT_FP4_RAZER ? 2 : 0);
+};
+struct MetaWin { long a0, a1, b0, b1, bpl; };
+template <int FMT>
+__host__ __device__ inline MetaWin meta_window(long r_lo, long r_hi, long GK, long z0, long rows_cap) {
+  using MP = MetaPlanes<FMT>;
+  MetaWin m;
+  m.a0 = (MP::A * r_lo * GK) & ~15L;
+  m.a1 = (MP::A * r_hi * GK + 15) & ~15L;
+  m.bpl = (MP::A * rows_cap * GK + 32 + 15) & ~15L;   // plane B's offset in the staged copy
+  if (MP::B) {
+    m.b0 = (z0 + (r_lo * GK * MP::B) / 8) & ~15L;
+    m.b1 = (z0 + (r_hi * GK * MP::B + 7) / 8 + 15) & ~15L;
+  } else {
+    m.b0 = m.b1 = 0;
+  }
+  return m;
+}
+template <int FMT>
+__host__ __device__ inline size_t meta_stage_bytes(long rows_cap, long GK) {
+  using MP = MetaPlanes<FMT>;
+  const size_t a = ((size_t)MP::A * rows_cap * GK + 32 + 15) & ~size_t(15);
+  return a + (MP::B ? ((((size_t)rows_cap * GK * MP::B + 7) / 8 + 48 + 15) & ~size_t(15)) : 0);
+}
+// Metadata of group f from the staged copy.
+template <int FMT>
+__device__ __forceinline__ GroupMeta group_meta_s(const uint8_t* ms, const MetaWin& w, long z0, long f) {
+  GroupMeta g;
+  if (FMT == QNT_FP4_AFPQ) {
+    const uint32_t v = lds_u32(ms + (4 * f - w.a0));
+    g.s = h2f(v & 0xFFFFu);
+    g.t = h2f(v >> 16);
+    return g;
+  }
+  const float s = h2f(lds_u16(ms + (2 * f - w.a0)));
+  if (FMT == QNT_INT4_ASYM) {
+    const uint32_t z = (lds_u8(ms + w.bpl + (z0 + f / 2 - w.b0)) >> (4 * (f & 1))) & 15u;
+    g.s = s * 16777216.0f;
+    g.t = s * (float)z;
+  } else if (FMT == QNT_FP4_RAZER) {
+    const uint32_t sel = (lds_u8(ms + w.bpl + (z0 + f / 4 - w.b0)) >> (2 * (f & 3))) & 3u;
+    const float sv = (sel & 2u) ? 8.0f : 5.0f;
+    g.s = s;
+    g.t = (sel & 1u) ? -sv : sv;
+  } else {
+    g.s = s;
+    g.t = 0.0f;
+  }
+  return g;
+}
+
 // ------------------------------------------------------------------ per-chunk dot products
 // One 16-byte chunk c of a 4-bit row (32 weights, order as in the layout) with
 // the activations xk of its first weight.  acc[0..3]: INT4 [0,1] nibbles at bit
@@ -194,14 +250,17 @@ __host__ __device__ inline int simt_ranges(int fmt, int K) {
 }
 
 // Shared-memory carve-up (byte offsets), used by the kernel and the launcher.
-struct SmemSimt { size_t xs, xg, part, total; };
-__host__ __device__ inline SmemSimt smem_simt_layout(int fmt, int MB, int K, int group, int rows_cap) {
+struct SmemSimt { size_t xs, xg, part, ms, total; };
+// meta_bytes: size of the staged metadata copy (0: read from global memory)
+__host__ __device__ inline SmemSimt smem_simt_layout(int fmt, int MB, int K, int group, int rows_cap,
+                                                      size_t meta_bytes) {
   const int KR = simt_ranges(fmt, K);
   SmemSimt L;
   L.xs = (size_t)kCtrlBytes + kRingBytes;
   L.xg = align16(L.xs + (size_t)MB * K * 2);
   L.part = align16(L.xg + (fmt == QNT_INT4_ASYM ? (size_t)MB * (K / group) * 4 : 0));
-  L.total = align16(L.part + (size_t)MB * rows_cap * KR * 4);
+  L.ms = align16(L.part + (size_t)MB * rows_cap * KR * 4);
+  L.total = align16(L.ms + meta_bytes);
   return L;
 }
 
@@ -224,7 +283,7 @@ template <int FMT, int G, int MB>
 __global__ void __launch_bounds__(kThreads, 1)
 gemv_simt_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ meta, long z0,
                  const void* __restrict__ X, void* __restrict__ Y, int N, int K, int ldy, int xbf16,
-                 int rows_cap, int* d_status) {
+                 int rows_cap, int meta_bytes, int* d_status) {
   constexpr bool Q4 = FMT != QNT_INT8_PERCHAN && FMT != QNT_FP16;
   constexpr int WPC = FMT == QNT_INT8_PERCHAN ? 16 : 8;   // weights per 16-byte chunk (INT8 / FP16)
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -232,10 +291,11 @@ gemv_simt_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ 
   uint64_t* rbar = reinterpret_cast<uint64_t*>(smem + 64);
   float* red = reinterpret_cast<float*>(smem + 512);
   uint8_t* ring = smem + kCtrlBytes;
-  const SmemSimt L = smem_simt_layout(FMT, MB, K, Q4 ? G : K, rows_cap);
+  const SmemSimt L = smem_simt_layout(FMT, MB, K, Q4 ? G : K, rows_cap, (size_t)meta_bytes);
   __half* xs = reinterpret_cast<__half*>(smem + L.xs);
   float* xg = reinterpret_cast<float*>(smem + L.xg);         // [MB][K/G] group sums (INT4)
   float* part = reinterpret_cast<float*>(smem + L.part);     // [MB][rows_cap][KR]
+  uint8_t* ms = smem + L.ms;                                  // staged metadata (4-bit formats)
   const long rowbytes = FMT == QNT_INT8_PERCHAN ? (long)K : 2L * K;   // INT8 / FP16
   const int KR = simt_ranges(FMT, K);
   const int GK = Q4 ? K / G : 1;
@@ -249,13 +309,27 @@ gemv_simt_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ 
   uint64_t* mybar = rbar + warp * kStages;
   uint8_t* myring = ring + (size_t)warp * kStages * kItemBytes;
 
-  if (tid == 0) mbar_init(xbar, 1);
+  if (tid == 0) {
+    mbar_init(xbar, 1);
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  }
   if (lane == 0)
     for (int s = 0; s < kStages; ++s) mbar_init(mybar + s, 1);
   __syncthreads();
+  MetaWin mw = {0, 0, 0, 0, 0};
+  if (Q4) mw = meta_window<Q4 ? FMT : QNT_FP4_E2M1>(r_lo, r_hi, GK, z0, rows_cap);
   if (tid == 0) {
     const uint32_t xbytes = (uint32_t)K * 2u;
-    mbar_expect_tx(xbar, xbytes * MB);
+    const bool stage_meta = Q4 && meta_bytes > 0 && r_hi > r_lo;
+    mbar_expect_tx(xbar, xbytes * MB + (stage_meta ? (uint32_t)((mw.a1 - mw.a0) + (mw.b1 - mw.b0)) : 0u));
+    if (stage_meta) {
+      bulk_g2s(ms, meta + mw.a0, (uint32_t)(mw.a1 - mw.a0), xbar);
+      if (mw.b1 > mw.b0) bulk_g2s(ms + mw.bpl, meta + mw.b0, (uint32_t)(mw.b1 - mw.b0), xbar);
+    }
+    // programmatic dependent launch: the activations (and, after them, every
+    // write of Y) wait for the previous kernel in the stream; weights and
+    // metadata, which no kernel of this library writes, are already requested
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     for (int m = 0; m < MB; ++m)
       bulk_g2s(xs + (size_t)m * K, static_cast<const uint8_t*>(X) + (size_t)m * xbytes, xbytes, xbar);
   }
@@ -307,28 +381,38 @@ gemv_simt_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ 
     if (!mbar_wait(mybar + stage, phase)) { failed = true; break; }
     const uint8_t* st = myring + (size_t)stage * kItemBytes;
     if (Q4) {
-      // lane l: row i8 = l/4 of the group, chunk position l%4 of every block
-      const int i8 = lane >> 2, up = lane & 3;
-      const int cu = up ^ ((i8 >> 1) & 3);                   // chunk held at that position
+      // lane l: row i8 = l % 8 of the group, blocks hq = l / 8 and hq + 4 of the
+      // range (whole 128-weight blocks, so a G = 128 group is one lane's); the
+      // eight lanes of a shared-memory phase read one chunk of eight rows
+      // (conflict-free by the layout's swizzle) and the same activations
+      const int i8 = lane & 7, hq = lane >> 3;
       const long row = r_lo + 8 * un + i8;
       const int nblk = min(8, K / 128 - 8 * kr);
       float acc[MB];
 #pragma unroll
       for (int m = 0; m < MB; ++m) acc[m] = 0.0f;
-#pragma unroll 2
-      for (int h = 0; h < nblk; ++h) {
-        const uint4 v = lds128(st + 512 * h + 64 * i8 + 16 * up);
-        const long k0 = (long)kr * kRange4 + 128 * h + 32 * cu;   // first weight of the chunk
-        GroupMeta md = {0.0f, 0.0f};
-        if (row < r_hi) md = group_meta<FMT>(meta, z0, row * GK + k0 / G);
 #pragma unroll
-        for (int m = 0; m < MB; ++m) {
-          float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-          float corr = 0.0f;
-          dot_chunk4<FMT>(v, xs + (size_t)m * K + k0, a, corr);
-          float val = chunk_value<FMT>(md, a, corr);
-          if (FMT == QNT_INT4_ASYM && (k0 % G) == 0) val -= md.t * xg[(size_t)m * GK + k0 / G];
-          acc[m] += val;
+      for (int hh = 0; hh < 2; ++hh) {
+        const int h = hq + 4 * hh;
+        if (h < nblk) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 v = lds128(st + 512 * h + 64 * i8 + 16 * (c ^ ((i8 >> 1) & 3)));
+            const long k0 = (long)kr * kRange4 + 128 * h + 32 * c;   // first weight of the chunk
+            GroupMeta md = {0.0f, 0.0f};
+            if (row < r_hi)
+              md = meta_bytes > 0 ? group_meta_s<FMT>(ms, mw, z0, row * GK + k0 / G)
+                                  : group_meta<FMT>(meta, z0, row * GK + k0 / G);
+#pragma unroll
+            for (int m = 0; m < MB; ++m) {
+              float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+              float corr = 0.0f;
+              dot_chunk4<FMT>(v, xs + (size_t)m * K + k0, a, corr);
+              float val = chunk_value<FMT>(md, a, corr);
+              if (FMT == QNT_INT4_ASYM && (k0 % G) == 0) val -= md.t * xg[(size_t)m * GK + k0 / G];
+              acc[m] += val;
+            }
+          }
         }
       }
       __syncwarp();
@@ -339,9 +423,9 @@ gemv_simt_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ 
 #pragma unroll
       for (int m = 0; m < MB; ++m) {
         float y4 = acc[m];
-        y4 += __shfl_xor_sync(0xffffffffu, y4, 1);
-        y4 += __shfl_xor_sync(0xffffffffu, y4, 2);
-        if (up == 0 && row < r_hi) part[((size_t)m * rows_cap + (row - r_lo)) * KR + kr] = y4;
+        y4 += __shfl_xor_sync(0xffffffffu, y4, 8);
+        y4 += __shfl_xor_sync(0xffffffffu, y4, 16);
+        if (hq == 0 && row < r_hi) part[((size_t)m * rows_cap + (row - r_lo)) * KR + kr] = y4;
       }
       continue;
     }
@@ -432,6 +516,268 @@ gemv_simt_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ 
   }
 }
 
+// ------------------------------------------------------------------ 4-bit kernel, one vector
+// Batch 1 keeps each lane's activations in registers.  Lane l owns block l
+// (128 weights) of a 32-block range of K: its 128 activations (64 registers),
+// and for INT4 its group sums, are loaded once per range.  A work item is one
+// row group (8 rows) x one range, a contiguous 16 KB run of the packed layout
+// fetched with one bulk copy into a CTA-wide ring by a producer warp.  In step
+// `it` of an item, lane l processes row (l + it) % 8 of the group: the eight
+// lanes of a shared-memory phase then read one chunk of eight different rows,
+// which the layout's chunk swizzle spreads over eight bank groups.  Per-row
+// partial sums are folded across lanes with shuffles and combined across
+// ranges in a fixed order.
+constexpr int kRgConsumers = 7;
+constexpr int kRgThreads = 32 * (1 + kRgConsumers);
+constexpr int kRgLanesBlocks = 32;                        // blocks per range
+constexpr int kRgItemBytes = 8 * kRgLanesBlocks * 64;     // 16 KB
+constexpr int kRgMaxSlots = 8;
+constexpr int kRgCtrl = 1024;
+
+struct SmemRg { size_t ring, xs, part, ms, total; };
+__host__ __device__ inline SmemRg smem_rg_layout(int K, int rows_cap, int nslot, size_t meta_bytes) {
+  const int KBR = (K / 128 + kRgLanesBlocks - 1) / kRgLanesBlocks;
+  SmemRg L;
+  L.ring = kRgCtrl;
+  L.xs = L.ring + (size_t)nslot * kRgItemBytes;
+  L.part = align16(L.xs + (size_t)K * 2);
+  L.ms = align16(L.part + (size_t)rows_cap * KBR * 4);
+  L.total = align16(L.ms + meta_bytes);
+  return L;
+}
+
+// x of this lane's block: 16 uint4 of fp16 (bf16 inputs scaled by 2^e into fp16
+// range, exactly; inv = 2^-e undoes it), INT4 group sums of the unscaled values.
+template <int FMT, int G>
+__device__ __forceinline__ void rg_load_x(const uint8_t* xs, long b, int KB, int xbf16, uint4 (&xr)[16],
+                                          float (&xgs)[128 / G], float& inv) {
+  constexpr int GPB = 128 / G;
+#pragma unroll
+  for (int q = 0; q < GPB; ++q) xgs[q] = 0.0f;
+  inv = 1.0f;
+  if (b >= KB) {
+#pragma unroll
+    for (int u = 0; u < 16; ++u) xr[u] = make_uint4(0, 0, 0, 0);
+    return;
+  }
+  const uint8_t* src = xs + b * 256;
+#pragma unroll
+  for (int u = 0; u < 16; ++u) xr[u] = lds128(src + 16 * u);
+  if (xbf16) {
+    float am = 0.0f;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const uint32_t w[4] = {xr[u].x, xr[u].y, xr[u].z, xr[u].w};
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        am = fmaxf(am, fabsf(__uint_as_float(w[p] << 16)));
+        am = fmaxf(am, fabsf(__uint_as_float(w[p] & 0xFFFF0000u)));
+      }
+    }
+    int e = 0;
+    if (am > 0.0f && isfinite(am)) e = min(max(14 - (int)((__float_as_uint(am) >> 23) & 255u) + 127, -126), 126);
+    const float f = __uint_as_float((uint32_t)(127 + e) << 23);
+    inv = __uint_as_float((uint32_t)(127 - e) << 23);
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      uint32_t w[4] = {xr[u].x, xr[u].y, xr[u].z, xr[u].w};
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const float lo = __uint_as_float(w[p] << 16), hi = __uint_as_float(w[p] & 0xFFFF0000u);
+        if (FMT == QNT_INT4_ASYM) xgs[(8 * u) / G] += lo + hi;
+        const __half2 h = __floats2half2_rn(lo * f, hi * f);
+        w[p] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      xr[u] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  } else if (FMT == QNT_INT4_ASYM) {
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const uint32_t w[4] = {xr[u].x, xr[u].y, xr[u].z, xr[u].w};
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&w[p]));
+        xgs[(8 * u) / G] += f2.x + f2.y;
+      }
+    }
+  }
+}
+
+template <int FMT, int G>
+__global__ void __launch_bounds__(kRgThreads, 1)
+gemv4_rg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ meta, long z0,
+                const void* __restrict__ X, void* __restrict__ Y, int N, int K, int xbf16, int rows_cap,
+                int nslot, int meta_bytes, int* d_status) {
+  constexpr int GPB = 128 / G;              // groups per block
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + kRgMaxSlots;
+  uint64_t* xbar = empty + kRgMaxSlots;
+  volatile int* abort_p = reinterpret_cast<volatile int*>(smem + 512);
+  const SmemRg L = smem_rg_layout(K, rows_cap, nslot, (size_t)meta_bytes);
+  uint8_t* ring = smem + L.ring;
+  uint8_t* xs = smem + L.xs;
+  float* part = reinterpret_cast<float*>(smem + L.part);    // [rows_cap][KBR]
+  uint8_t* ms = smem + L.ms;
+  const int KB = K / 128, KBR = (KB + kRgLanesBlocks - 1) / kRgLanesBlocks, GK = K / G;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  long r_lo, r_hi;
+  simt_rows(QNT_INT4_ASYM, N, blockIdx.x, gridDim.x, &r_lo, &r_hi);
+  const int nrows = (int)(r_hi - r_lo);
+  const int nitems = (nrows + 7) / 8 * KBR;
+  const MetaWin mw = meta_window<FMT>(r_lo, r_hi, GK, z0, rows_cap);
+
+  if (tid == 0) {
+    for (int i = 0; i < nslot; ++i) { mbar_init(full + i, 1); mbar_init(empty + i, 1); }
+    mbar_init(xbar, 1);
+    *abort_p = 0;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      const uint64_t pol = l2_evict_first_policy();
+      auto issue = [&](int t) {
+        const int u = t / KBR, br = t - u * KBR, slot = t % nslot;
+        const int nb = min(kRgLanesBlocks, KB - kRgLanesBlocks * br);
+        mbar_expect_tx(full + slot, (uint32_t)nb * 512u);
+        bulk_g2s_hint(ring + (size_t)slot * kRgItemBytes, codes + (r_lo / 8 + u) * 4L * K + (long)br * kRgLanesBlocks * 512,
+                      (uint32_t)nb * 512u, full + slot, pol);
+      };
+      const bool stage_meta = meta_bytes > 0 && nrows > 0;
+      mbar_expect_tx(xbar, (uint32_t)K * 2u + (stage_meta ? (uint32_t)((mw.a1 - mw.a0) + (mw.b1 - mw.b0)) : 0u));
+      if (stage_meta) {
+        bulk_g2s(ms, meta + mw.a0, (uint32_t)(mw.a1 - mw.a0), xbar);
+        if (mw.b1 > mw.b0) bulk_g2s(ms + mw.bpl, meta + mw.b0, (uint32_t)(mw.b1 - mw.b0), xbar);
+      }
+      int t = 0;
+      for (; t < nitems && t < nslot; ++t) issue(t);   // weights do not depend on the previous kernel
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      bulk_g2s(xs, X, (uint32_t)K * 2u, xbar);
+      for (; t < nitems; ++t) {
+        if (!mbar_wait(empty + t % nslot, (uint32_t)(t / nslot - 1) & 1u)) {
+          *abort_p = 1;
+          report(d_status, QNT_ERR_TIMEOUT);
+          break;
+        }
+        issue(t);
+      }
+      // drain: every issued copy has landed before the CTA exits
+      mbar_wait(xbar, 0);
+      for (int i = (t > nslot ? t - nslot : 0); i < t; ++i) mbar_wait(full + i % nslot, (uint32_t)(i / nslot) & 1u);
+    }
+  } else {
+    // ---------------------------------------------------------------- consumers
+    const int cw = warp - 1;
+    if (!mbar_wait(xbar, 0)) { *abort_p = 1; report(d_status, QNT_ERR_TIMEOUT); }
+    uint4 xr[16];
+    float xgs[GPB];
+    float inv = 1.0f;
+    int cur_br = -1;
+    for (int t = cw; t < nitems && !*abort_p; t += kRgConsumers) {
+      const int u = t / KBR, br = t - u * KBR, slot = t % nslot;
+      const long b = (long)br * kRgLanesBlocks + lane;            // this lane's block
+      if (br != cur_br) { rg_load_x<FMT, G>(xs, b, KB, xbf16, xr, xgs, inv); cur_br = br; }
+      if (!mbar_wait(full + slot, (uint32_t)(t / nslot) & 1u)) { *abort_p = 1; report(d_status, QNT_ERR_TIMEOUT); break; }
+      const uint8_t* st = ring + (size_t)slot * kRgItemBytes + (size_t)lane * 512;
+      const bool has = b < KB;
+      float yit[8];
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        yit[it] = 0.0f;
+        const int i8 = (lane + it) & 7;
+        const long row = r_lo + 8 * u + i8;
+        if (!has || row >= r_hi) continue;
+#pragma unroll
+        for (int q = 0; q < GPB; ++q) {
+          const long f = row * GK + b * GPB + q;
+          const GroupMeta md = meta_bytes > 0 ? group_meta_s<FMT>(ms, mw, z0, f) : group_meta<FMT>(meta, z0, f);
+          float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          const float corr = 0.0f;   // RaZeR special values are placed in the decoded operands
+          uint32_t sv16 = 0;
+          if (FMT == QNT_FP4_RAZER) sv16 = __half_as_ushort(__float2half_rn(md.t));   // +-5 or +-8, exact
+#pragma unroll
+          for (int cc = 0; cc < 4 / GPB; ++cc) {
+            const int c = q * (4 / GPB) + cc;                  // chunk of the block
+            const uint4 cv = lds128(st + 64 * i8 + 16 * (c ^ ((i8 >> 1) & 3)));
+            const uint32_t w[4] = {cv.x, cv.y, cv.z, cv.w};
+#pragma unroll
+            for (int jw = 0; jw < 4; ++jw) {
+              if (FMT == QNT_INT4_ASYM) {
+                // word jw: low nibbles -> chunk weights 4jw..4jw+3, high -> 16+4jw..16+4jw+3
+                const uint4 xa = xr[4 * c + jw / 2], xb = xr[4 * c + 2 + jw / 2];
+                const uint32_t xl0 = (jw & 1) ? xa.z : xa.x, xl1 = (jw & 1) ? xa.w : xa.y;
+                const uint32_t xh0 = (jw & 1) ? xb.z : xb.x, xh1 = (jw & 1) ? xb.w : xb.y;
+                const uint32_t w8 = w[jw] >> 8;
+                fma_mixed2(w[jw] & 0x000F000Fu, xl0, a[0], a[1]);
+                fma_mixed2(w8 & 0x000F000Fu, xl1, a[0], a[1]);
+                fma_mixed2(w[jw] & 0x00F000F0u, xh0, a[2], a[3]);
+                fma_mixed2(w8 & 0x00F000F0u, xh1, a[2], a[3]);
+              } else {
+                const uint4 x4 = xr[4 * c + jw];                // chunk weights 8jw..8jw+7
+                uint32_t h[4];
+                cvt_e2m1x8(w[jw], h[0], h[1], h[2], h[3]);
+                if (FMT == QNT_FP4_AFPQ) {
+#pragma unroll
+                  for (int pp = 0; pp < 4; ++pp) {
+                    const uint32_t vp = hmax2(h[pp], 0u);
+                    const uint32_t vn = hsub2(h[pp], vp);
+                    fma_mixed2(vp, (&x4.x)[pp], a[0], a[1]);
+                    fma_mixed2(vn, (&x4.x)[pp], a[2], a[3]);
+                  }
+                } else {
+                  if (FMT == QNT_FP4_RAZER) {
+                    // weights coded 0b1000 (decoded as -0) take the group's special
+                    // value: nibble 2pp / 2pp+1 is the low / high half of h[pp]
+                    const uint32_t tt = (w[jw] & 0x77777777u) + 0x77777777u;
+                    const uint32_t spec = lop3<0x20>(w[jw], tt, 0x88888888u);
+                    if (spec) {
+#pragma unroll
+                      for (int pp = 0; pp < 4; ++pp) {
+                        if (spec & (0x8u << (8 * pp))) h[pp] = (h[pp] & 0xFFFF0000u) | sv16;
+                        if (spec & (0x80u << (8 * pp))) h[pp] = (h[pp] & 0x0000FFFFu) | (sv16 << 16);
+                      }
+                    }
+                  }
+#pragma unroll
+                  for (int pp = 0; pp < 4; ++pp) fma_mixed2(h[pp], (&x4.x)[pp], a[0], a[1]);
+                }
+              }
+            }
+          }
+          float v = chunk_value<FMT>(md, a, corr);
+          if (FMT == QNT_INT4_ASYM) v = v * inv - md.t * xgs[q];
+          else v *= inv;
+          yit[it] += v;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_addr(empty + slot)) : "memory");
+      // fold: lanes l, l+8, l+16, l+24 share rows; then lane r gathers row r
+      float tot = 0.0f;
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        float sv = yit[it];
+        sv += __shfl_xor_sync(0xffffffffu, sv, 8);
+        sv += __shfl_xor_sync(0xffffffffu, sv, 16);
+        tot += __shfl_sync(0xffffffffu, sv, (lane - it) & 7);   // lane (r - it) % 8 holds row r in step it
+      }
+      const long row = r_lo + 8 * u + lane;
+      if (lane < 8 && row < r_hi) part[(size_t)(8 * u + lane) * KBR + br] = tot;
+    }
+  }
+  __syncthreads();
+  for (int rl = tid; rl < nrows; rl += kRgThreads) {
+    float v = 0.0f;
+    for (int br = 0; br < KBR; ++br) v += part[(size_t)rl * KBR + br];
+    if (xbf16) reinterpret_cast<__nv_bfloat16*>(Y)[r_lo + rl] = __float2bfloat16_rn(v);
+    else reinterpret_cast<__half*>(Y)[r_lo + rl] = __float2half_rn(v);
+  }
+}
+
 // ------------------------------------------------------------------ launchers
 int num_sms() {
   static int sms[64] = {0};
@@ -473,22 +819,55 @@ static int simt_grid(const qnt_desc& d) {
   return units < num_sms() ? units : num_sms();
 }
 
-size_t gemv_smem_bytes(const qnt_desc& d, int MB, int grid) {
-  return smem_simt_layout(d.fmt, MB, d.K, d.group, simt_rows_cap(d, grid)).total;
+static size_t simt_meta_bytes(const qnt_desc& d, int rows_cap) {
+  const long GK = d.K / d.group;
+  switch (d.fmt) {
+    case QNT_INT4_ASYM: return meta_stage_bytes<QNT_INT4_ASYM>(rows_cap, GK);
+    case QNT_FP4_E2M1: return meta_stage_bytes<QNT_FP4_E2M1>(rows_cap, GK);
+    case QNT_FP4_AFPQ: return meta_stage_bytes<QNT_FP4_AFPQ>(rows_cap, GK);
+    case QNT_FP4_RAZER: return meta_stage_bytes<QNT_FP4_RAZER>(rows_cap, GK);
+    default: return 0;
+  }
 }
+
+// Shared memory of a launch; *meta_bytes: the staged metadata copy, or 0 when
+// it would not fit (the kernel then reads metadata from global memory).
+static size_t simt_smem(const qnt_desc& d, int MB, int grid, size_t* meta_bytes) {
+  const int rows_cap = simt_rows_cap(d, grid);
+  size_t mb = simt_meta_bytes(d, rows_cap);
+  size_t total = smem_simt_layout(d.fmt, MB, d.K, d.group, rows_cap, mb).total;
+  if (total > (size_t)kMaxDynSmem) {
+    mb = 0;
+    total = smem_simt_layout(d.fmt, MB, d.K, d.group, rows_cap, 0).total;
+  }
+  if (meta_bytes) *meta_bytes = mb;
+  return total;
+}
+
+size_t gemv_smem_bytes(const qnt_desc& d, int MB, int grid) { return simt_smem(d, MB, grid, nullptr); }
 
 template <int FMT, int G, int MB>
 static cudaError_t launch_simt(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
                                int ldy, int xbf16, int* st, cudaStream_t s) {
   const int grid = simt_grid(d);
-  const size_t smem = gemv_smem_bytes(d, MB, grid);
+  size_t meta_bytes = 0;
+  const size_t smem = simt_smem(d, MB, grid, &meta_bytes);
   auto kfn = gemv_simt_kernel<FMT, G, MB>;
   cudaError_t e = configure_smem(reinterpret_cast<const void*>(kfn));
   if (e != cudaSuccess) return e;
   const int rows_cap = simt_rows_cap(d, grid);
-  kfn<<<grid, kThreads, smem, s>>>(static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(meta), z0, X, Y,
-                                   d.N, d.K, ldy, xbf16, rows_cap, st);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kfn, static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(meta), z0, X, Y,
+                            d.N, d.K, ldy, xbf16, rows_cap, (int)meta_bytes, st);
 }
 
 template <int MB>
@@ -519,6 +898,60 @@ int gemv_max_mb(const qnt_desc& d) {
   for (int mb : {1, 2, 4, 8})
     if (gemv_smem_bytes(d, mb, grid) <= (size_t)kMaxDynSmem) best = mb;
   return best;
+}
+
+template <int FMT, int G>
+static cudaError_t launch_rg(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
+                             int xbf16, int* st, cudaStream_t s, bool* handled) {
+  const int grid = simt_grid(d);
+  const int rows_cap = simt_rows_cap(d, grid);
+  size_t mb = meta_stage_bytes<FMT>(rows_cap, d.K / d.group);
+  int nslot = kRgMaxSlots;
+  while (nslot > 2 && smem_rg_layout(d.K, rows_cap, nslot, mb).total > (size_t)kMaxDynSmem) --nslot;
+  if (smem_rg_layout(d.K, rows_cap, nslot, mb).total > (size_t)kMaxDynSmem) {
+    mb = 0;   // metadata from global memory
+    nslot = kRgMaxSlots;
+    while (nslot > 2 && smem_rg_layout(d.K, rows_cap, nslot, 0).total > (size_t)kMaxDynSmem) --nslot;
+    if (smem_rg_layout(d.K, rows_cap, nslot, 0).total > (size_t)kMaxDynSmem) return cudaSuccess;   // not handled
+  }
+  const size_t smem = smem_rg_layout(d.K, rows_cap, nslot, mb).total;
+  auto kfn = gemv4_rg_kernel<FMT, G>;
+  cudaError_t e = configure_smem(reinterpret_cast<const void*>(kfn));
+  if (e != cudaSuccess) return e;
+  *handled = true;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kRgThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kfn, static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(meta), z0, X, Y,
+                            d.N, d.K, xbf16, rows_cap, nslot, (int)mb, st);
+}
+
+// One activation vector, 4-bit formats: the register-resident kernel above.
+// *handled = false when it does not take the shape.
+cudaError_t launch_gemv4_one(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
+                             int xbf16, int* st, cudaStream_t s, bool* handled) {
+  *handled = false;
+#define QNT_RG(FMT)                                                                          \
+  switch (d.group) {                                                                         \
+    case 32: return launch_rg<FMT, 32>(d, codes, meta, z0, X, Y, xbf16, st, s, handled);     \
+    case 64: return launch_rg<FMT, 64>(d, codes, meta, z0, X, Y, xbf16, st, s, handled);     \
+    default: return launch_rg<FMT, 128>(d, codes, meta, z0, X, Y, xbf16, st, s, handled);    \
+  }
+  switch (d.fmt) {
+    case QNT_INT4_ASYM: QNT_RG(QNT_INT4_ASYM)
+    case QNT_FP4_E2M1: QNT_RG(QNT_FP4_E2M1)
+    case QNT_FP4_AFPQ: QNT_RG(QNT_FP4_AFPQ)
+    case QNT_FP4_RAZER: QNT_RG(QNT_FP4_RAZER)
+    default: return cudaSuccess;
+  }
+#undef QNT_RG
 }
 
 // Y[m] = W x[m] for m < M on CUDA cores, in passes of up to 8 vectors.

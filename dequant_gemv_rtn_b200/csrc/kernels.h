@@ -22,6 +22,11 @@ cudaError_t launch_quantize(const qnt_desc& d, const float* W, void* codes, void
 cudaError_t launch_gemv_simt(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X,
                              void* Y, int M, int xbf16, int* st, cudaStream_t s);
 
+// y = W x for one activation vector, 4-bit formats, on CUDA cores with the
+// activations in registers (gemv.cu).  *handled = false when it does not apply.
+cudaError_t launch_gemv4_one(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
+                             int xbf16, int* st, cudaStream_t s, bool* handled);
+
 // Y[m] = W x[m] for m < M on the tensor cores (gemv_tc.cu).  Returns with
 // *handled = false, launching nothing, when the tensor-core kernel does not
 // take this format / batch / shape.

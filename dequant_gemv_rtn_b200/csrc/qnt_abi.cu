@@ -35,19 +35,33 @@ int check(const qnt_desc* d) {
   return QNT_OK;
 }
 
-// Y[m] = W x[m], m < M: the tensor-core kernel where it applies, else the
-// CUDA-core kernel.  QNT_FORCE_SIMT=1 in the environment selects the CUDA-core
-// kernel everywhere (used to test both paths on the same inputs).
+// Y[m] = W x[m], m < M.  Kernel choice (measured on B200 with L2-cold weights,
+// 14336 x 4096 and the Llama-7B decode shapes):
+//   one vector, INT4 / FP4 / AFPQ   -> register-resident CUDA-core kernel
+//   INT4 2..8 vectors; FP4; AFPQ;
+//   RaZeR 1..2 vectors               -> CUDA-core multi-vector kernel
+//   INT4 9..16, RaZeR 3..16 vectors  -> tensor-core kernel (tcgen05)
+//   INT8, FP16, more than 16 vectors -> CUDA-core multi-vector kernel
+// QNT_FORCE_SIMT=1 selects the CUDA-core multi-vector kernel everywhere and
+// QNT_FORCE_TC=1 the tensor-core kernel wherever it applies (used to test every
+// path on the same inputs).
 cudaError_t dispatch_gemm(const qnt_desc& d, const void* codes, const void* meta, const void* X, void* Y, int M,
                           int xbf16, int* st, cudaStream_t s) {
-  static const bool force_simt = [] {
-    const char* v = std::getenv("QNT_FORCE_SIMT");
-    return v && v[0] == '1';
+  static const int force = [] {
+    const char* a = std::getenv("QNT_FORCE_SIMT");
+    const char* b = std::getenv("QNT_FORCE_TC");
+    return (a && a[0] == '1') ? 1 : ((b && b[0] == '1') ? 2 : 0);
   }();
   const long z0 = zero_plane(d);
-  if (!force_simt) {
-    bool handled = false;
-    cudaError_t e = qnt::launch_gemv_tc(d, codes, meta, z0, X, Y, M, xbf16, st, s, &handled);
+  bool handled = false;
+  cudaError_t e = cudaSuccess;
+  if (force == 0 && M == 1 && d.fmt != QNT_FP4_RAZER) {
+    e = qnt::launch_gemv4_one(d, codes, meta, z0, X, Y, xbf16, st, s, &handled);
+    if (handled || e != cudaSuccess) return e;
+  }
+  const bool tc = force == 2 || (force == 0 && ((d.fmt == QNT_INT4_ASYM && M > 8) || (d.fmt == QNT_FP4_RAZER && M > 2)));
+  if (tc) {
+    e = qnt::launch_gemv_tc(d, codes, meta, z0, X, Y, M, xbf16, st, s, &handled);
     if (handled || e != cudaSuccess) return e;
   }
   return qnt::launch_gemv_simt(d, codes, meta, z0, X, Y, M, xbf16, st, s);

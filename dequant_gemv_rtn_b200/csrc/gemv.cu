@@ -527,12 +527,13 @@ gemv_simt_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ 
 // which the layout's chunk swizzle spreads over eight bank groups.  Per-row
 // partial sums are folded across lanes with shuffles and combined across
 // ranges in a fixed order.
-constexpr int kRgConsumers = 7;
+constexpr int kRgConsumers = 3;                           // 128-thread CTAs: two fit an SM
 constexpr int kRgThreads = 32 * (1 + kRgConsumers);
 constexpr int kRgLanesBlocks = 32;                        // blocks per range
 constexpr int kRgItemBytes = 8 * kRgLanesBlocks * 64;     // 16 KB
 constexpr int kRgMaxSlots = 8;
 constexpr int kRgCtrl = 1024;
+constexpr int kRgSmemCap = 113 * 1024;                    // leaves room for a second CTA
 
 struct SmemRg { size_t ring, xs, part, ms, total; };
 __host__ __device__ inline SmemRg smem_rg_layout(int K, int rows_cap, int nslot, size_t meta_bytes) {
@@ -603,6 +604,24 @@ __device__ __forceinline__ void rg_load_x(const uint8_t* xs, long b, int KB, int
   }
 }
 
+// Wait until ring slot `slot` holds item t and its bytes have landed.  The tag
+// is read first: the producer writes t there only after the slot's previous
+// item has been consumed, so from then on the slot barrier's pending (or last
+// completed) phase is the one for t, and the parity wait cannot be met by a
+// phase two behind.  Bounded like every wait; false on timeout or abort.
+__device__ __forceinline__ bool rg_wait_item(volatile int* tag, uint64_t* full, int slot, int t, int nslot,
+                                             volatile int* abort_p) {
+  for (int it = 0; it < kMaxTries; ++it) {
+    if (tag[slot] == t) {
+      __threadfence_block();
+      return mbar_wait(full + slot, (uint32_t)(t / nslot) & 1u);
+    }
+    if (*abort_p) return false;
+    __nanosleep(256);
+  }
+  return false;
+}
+
 template <int FMT, int G>
 __global__ void __launch_bounds__(kRgThreads, 1)
 gemv4_rg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ meta, long z0,
@@ -614,6 +633,9 @@ gemv4_rg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ m
   uint64_t* empty = full + kRgMaxSlots;
   uint64_t* xbar = empty + kRgMaxSlots;
   volatile int* abort_p = reinterpret_cast<volatile int*>(smem + 512);
+  // item last issued into each slot: consumers share the ring, so one may come
+  // to an item while its slot still holds an older one (see rg_wait_item)
+  volatile int* tag = reinterpret_cast<volatile int*>(smem + 640);
   const SmemRg L = smem_rg_layout(K, rows_cap, nslot, (size_t)meta_bytes);
   uint8_t* ring = smem + L.ring;
   uint8_t* xs = smem + L.xs;
@@ -629,7 +651,7 @@ gemv4_rg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ m
   const MetaWin mw = meta_window<FMT>(r_lo, r_hi, GK, z0, rows_cap);
 
   if (tid == 0) {
-    for (int i = 0; i < nslot; ++i) { mbar_init(full + i, 1); mbar_init(empty + i, 1); }
+    for (int i = 0; i < nslot; ++i) { mbar_init(full + i, 1); mbar_init(empty + i, 1); tag[i] = -1; }
     mbar_init(xbar, 1);
     *abort_p = 0;
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -643,6 +665,7 @@ gemv4_rg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ m
       auto issue = [&](int t) {
         const int u = t / KBR, br = t - u * KBR, slot = t % nslot;
         const int nb = min(kRgLanesBlocks, KB - kRgLanesBlocks * br);
+        tag[slot] = t;   // before the arrive below, which releases it to the waiters
         mbar_expect_tx(full + slot, (uint32_t)nb * 512u);
         bulk_g2s_hint(ring + (size_t)slot * kRgItemBytes, codes + (r_lo / 8 + u) * 4L * K + (long)br * kRgLanesBlocks * 512,
                       (uint32_t)nb * 512u, full + slot, pol);
@@ -681,7 +704,7 @@ gemv4_rg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ m
       const int u = t / KBR, br = t - u * KBR, slot = t % nslot;
       const long b = (long)br * kRgLanesBlocks + lane;            // this lane's block
       if (br != cur_br) { rg_load_x<FMT, G>(xs, b, KB, xbf16, xr, xgs, inv); cur_br = br; }
-      if (!mbar_wait(full + slot, (uint32_t)(t / nslot) & 1u)) { *abort_p = 1; report(d_status, QNT_ERR_TIMEOUT); break; }
+      if (!rg_wait_item(tag, full, slot, t, nslot, abort_p)) { *abort_p = 1; report(d_status, QNT_ERR_TIMEOUT); break; }
       const uint8_t* st = ring + (size_t)slot * kRgItemBytes + (size_t)lane * 512;
       const bool has = b < KB;
       float yit[8];
@@ -903,16 +926,25 @@ int gemv_max_mb(const qnt_desc& d) {
 template <int FMT, int G>
 static cudaError_t launch_rg(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
                              int xbf16, int* st, cudaStream_t s, bool* handled) {
-  const int grid = simt_grid(d);
-  const int rows_cap = simt_rows_cap(d, grid);
+  // two CTAs per SM: the row groups are split over twice the SM count, and a CTA
+  // small enough to share its SM lets the next kernel's CTAs start early
+  const int NG = (d.N + 7) / 8;
+  const int grid = NG < 2 * num_sms() ? NG : 2 * num_sms();
+  const int rows_cap = 8 * ((NG + grid - 1) / grid);
   size_t mb = meta_stage_bytes<FMT>(rows_cap, d.K / d.group);
   int nslot = kRgMaxSlots;
-  while (nslot > 2 && smem_rg_layout(d.K, rows_cap, nslot, mb).total > (size_t)kMaxDynSmem) --nslot;
-  if (smem_rg_layout(d.K, rows_cap, nslot, mb).total > (size_t)kMaxDynSmem) {
+  size_t cap = kRgSmemCap;
+  while (nslot > 2 && smem_rg_layout(d.K, rows_cap, nslot, mb).total > cap) --nslot;
+  if (smem_rg_layout(d.K, rows_cap, nslot, mb).total > cap) {   // alone on its SM, then
+    cap = kMaxDynSmem;
+    nslot = kRgMaxSlots;
+    while (nslot > 2 && smem_rg_layout(d.K, rows_cap, nslot, mb).total > cap) --nslot;
+  }
+  if (smem_rg_layout(d.K, rows_cap, nslot, mb).total > cap) {
     mb = 0;   // metadata from global memory
     nslot = kRgMaxSlots;
-    while (nslot > 2 && smem_rg_layout(d.K, rows_cap, nslot, 0).total > (size_t)kMaxDynSmem) --nslot;
-    if (smem_rg_layout(d.K, rows_cap, nslot, 0).total > (size_t)kMaxDynSmem) return cudaSuccess;   // not handled
+    while (nslot > 2 && smem_rg_layout(d.K, rows_cap, nslot, 0).total > cap) --nslot;
+    if (smem_rg_layout(d.K, rows_cap, nslot, 0).total > cap) return cudaSuccess;   // not handled
   }
   const size_t smem = smem_rg_layout(d.K, rows_cap, nslot, mb).total;
   auto kfn = gemv4_rg_kernel<FMT, G>;

@@ -53,7 +53,7 @@ STEP_BYTES = LAYERS * sum(algo_bytes_int4(N, K) for _, N, K in SHAPES)
 # the five shapes of a layer, from single-launch cold-cache ncu captures
 # (profiles/gemv4_rg_int4_g128_decode_shapes.md).  Set to None whenever the
 # kernel changes until it is captured again.
-TRAFFIC_PER_LAUNCH = 21122099
+TRAFFIC_PER_LAUNCH = None
 
 
 def measured_peaks():
@@ -293,7 +293,7 @@ def run_ours(args, world, rank, local):
         "roofline": {"bound": "hbm", "achieved": round(STEP_BYTES / launches / (step_ms * 1e-3 / launches) / 1e9, 1),
                      "peak": peak, "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy)" if peak_kind == "measured" else "fallback",
                      "unit": "GB/s", "frac": round(STEP_BYTES / (step_ms * 1e-3) / 1e9 / peak, 4),
-                     "traffic": TRAFFIC_PER_LAUNCH, "kernel": "gemv4_rg_kernel<INT4,g128>",
+                     "traffic": TRAFFIC_PER_LAUNCH, "kernel": "gemv4_mma_kernel<INT4,g128>",
                      "per_launch_bytes": STEP_BYTES // launches},
         "per_shape_isolated": per_shape,
         "gpu_launches": launches * args.steps,

@@ -801,6 +801,308 @@ gemv4_rg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ m
   }
 }
 
+// ------------------------------------------------------------------ batch 1 on the tensor cores (mma.sync)
+// The same producer ring as above, but the consumers hand the multiply-adds to
+// mma.sync m16n8k16 (fp16 inputs, fp32 accumulation) straight from the packed
+// layout, so a lane spends a handful of bit operations and one MMA on eight
+// weights instead of eight multiply-adds.
+//
+// One MMA covers the eight rows of a row group over 32 weights of each row.  Lane
+// t = 4g + r holds the 16-byte chunk r of row g of a block; word j of that chunk
+// feeds MMA j of the block.  A row g of the MMA's A operand is the row's first
+// half of the word's weights, row g + 8 its second half (two K segments of one
+// weight row); B column 2h + s holds the activations of segment s restricted to
+// group h of the block, so D[g][2h] + D[g + 8][2h + 1] is row g's dot product
+// over group h, found in lane 4g + h.  Which weights a word's halves hold is
+// fixed by the layout (INT4: nibbles at bits 0..3 and 4..7 of each fp16 half,
+// the latter 16x larger; FP4 family: e2m1 pairs), and the activation image
+// (xf, built once per CTA) puts each x where its weight's product lands.
+// Activations are scaled per block by an exact power of two that puts the block
+// maximum in [2^14, 2^15); B entries of INT4 nibbles at bits 4..7 carry x / 16.
+constexpr int kMmaConsumers = 7;
+constexpr int kMmaThreads = 32 * (1 + kMmaConsumers);
+constexpr int kMmaRangeBlocks = 8;                        // blocks per work item
+constexpr int kMmaItemBytes = kMmaRangeBlocks * 512;      // 4 KB: one row group x 8 blocks
+constexpr int kMmaMaxSlots = 24;
+constexpr int kMmaPrefetch = 4;                           // items requested before the activations
+constexpr int kMmaCtrl = 1024;                            // barriers, tags, 32 zero bytes at 768
+constexpr int kMmaSmemCap = 113 * 1024;                   // two CTAs per SM
+
+struct SmemMma { size_t ring, xraw, xf, xs2, part, ms, total; };
+__host__ __device__ inline SmemMma smem_mma_layout(int K, int G, int rows_cap, int nslot, size_t meta_bytes) {
+  const int KB = K / 128, KBR = (KB + kMmaRangeBlocks - 1) / kMmaRangeBlocks, GPB = 128 / G;
+  SmemMma L;
+  L.ring = kMmaCtrl;
+  L.xraw = L.ring + (size_t)nslot * kMmaItemBytes;
+  L.xf = align16(L.xraw + (size_t)K * 2);
+  L.xs2 = align16(L.xf + (size_t)K * 2);
+  L.part = align16(L.xs2 + (size_t)KB * GPB * 8);
+  L.ms = align16(L.part + (size_t)rows_cap * KBR * 4);
+  L.total = align16(L.ms + meta_bytes);
+  return L;
+}
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Byte offset in the activation image of the B entry for block b, chunk r,
+// segment s, MMA j, half hf (b0: hf = 0, b1: hf = 1).  A lane reads its
+// (s, r) entry of a block with two 16-byte loads (MMAs 0, 1 and 2, 3).
+__device__ __forceinline__ uint32_t xf_off(int b, int r, int s, int j, int hf) {
+  return (uint32_t)(256 * b + 128 * (j >> 1) + 16 * (4 * s + r) + 8 * (j & 1) + 4 * hf);
+}
+
+// Activation image of block b, built by one warp: lane l takes x[128b + 4l ..
+// 4l + 3].  Within a chunk, the weight at offset o = 16 hf + 4j + 2s + e (INT4)
+// or 8j + 4hf + 2s + e (FP4 family) meets B half hf, segment s of MMA j.  Also
+// writes (c / 2^e, sum of x over group h) per (block, group) to xs2, c = 2^24
+// for INT4 (undoes the subnormal encoding), else 1.
+template <int FMT, int G>
+__device__ __forceinline__ void mma_build_x(uint32_t xraw, uint32_t xf, uint32_t xs2, int b, int xbf16, int lane) {
+  constexpr int GPB = 128 / G;
+  const uint2 raw = lds64a(xraw + 256 * b + 8 * lane);
+  float v[4];
+  if (xbf16) {
+    v[0] = __uint_as_float(raw.x << 16); v[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(raw.y << 16); v[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+  } else {
+    v[0] = h2f(raw.x & 0xFFFFu); v[1] = h2f(raw.x >> 16);
+    v[2] = h2f(raw.y & 0xFFFFu); v[3] = h2f(raw.y >> 16);
+  }
+  float am = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+  float sgrp = (v[0] + v[1]) + (v[2] + v[3]);
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+    if (FMT == QNT_INT4_ASYM && o < G / 4) sgrp += __shfl_xor_sync(0xffffffffu, sgrp, o);
+  }
+  int e = 0;
+  if (am > 0.0f && isfinite(am)) e = min(max(14 - (int)((__float_as_uint(am) >> 23) & 255u) + 127, -126), 126);
+  const float f = __uint_as_float((uint32_t)(127 + e) << 23);
+  const int r = lane >> 3, o = 4 * (lane & 7);
+  int j, hf;
+  float fs = f;
+  if (FMT == QNT_INT4_ASYM) {
+    hf = o >> 4;
+    j = (o & 15) >> 2;
+    if (hf) fs = f * 0.0625f;   // these weights decode 16x too large
+  } else {
+    j = o >> 3;
+    hf = (o >> 2) & 1;
+  }
+  const __half2 p0 = __floats2half2_rn(v[0] * fs, v[1] * fs), p1 = __floats2half2_rn(v[2] * fs, v[3] * fs);
+  sts32a(xf + xf_off(b, r, 0, j, hf), *reinterpret_cast<const uint32_t*>(&p0));
+  sts32a(xf + xf_off(b, r, 1, j, hf), *reinterpret_cast<const uint32_t*>(&p1));
+  if ((lane & (G / 4 - 1)) == 0) {
+    const float inv = __uint_as_float((uint32_t)(127 - e) << 23) * (FMT == QNT_INT4_ASYM ? 16777216.0f : 1.0f);
+    sts64fa(xs2 + 8 * (b * GPB + lane / (G / 4)), inv, FMT == QNT_INT4_ASYM ? sgrp : 0.0f);
+  }
+}
+
+template <int FMT, int G>
+__global__ void __launch_bounds__(kMmaThreads, 2)
+gemv4_mma_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ meta, long z0,
+                 const void* __restrict__ X, void* __restrict__ Y, int N, int K, int xbf16, int rows_cap,
+                 int nslot, int meta_bytes, int* d_status) {
+  constexpr int GPB = 128 / G;
+  constexpr int RB = kMmaRangeBlocks;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + kMmaMaxSlots;
+  uint64_t* xbar = empty + kMmaMaxSlots;
+  volatile int* abort_p = reinterpret_cast<volatile int*>(smem + 512);
+  volatile int* tag = reinterpret_cast<volatile int*>(smem + 640);   // item last issued into each slot
+  const SmemMma L = smem_mma_layout(K, G, rows_cap, nslot, (size_t)meta_bytes);
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t zero_a = sbase + 768, ring_a = sbase + (uint32_t)L.ring, xraw_a = sbase + (uint32_t)L.xraw;
+  const uint32_t xf_a = sbase + (uint32_t)L.xf, xs2_a = sbase + (uint32_t)L.xs2;
+  uint8_t* ring = smem + L.ring;
+  float* part = reinterpret_cast<float*>(smem + L.part);    // [rows_cap][KBR]
+  uint8_t* ms = smem + L.ms;
+  const int KB = K / 128, KBR = (KB + RB - 1) / RB, GK = K / G;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  long r_lo, r_hi;
+  simt_rows(QNT_INT4_ASYM, N, blockIdx.x, gridDim.x, &r_lo, &r_hi);
+  const int nrows = (int)(r_hi - r_lo);
+  const int nitems = (nrows + 7) / 8 * KBR;
+  const MetaWin mw = meta_window<FMT>(r_lo, r_hi, GK, z0, rows_cap);
+
+  if (tid == 0) {
+    for (int i = 0; i < nslot; ++i) { mbar_init(full + i, 1); mbar_init(empty + i, 1); tag[i] = -1; }
+    mbar_init(xbar, 1);
+    *abort_p = 0;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  }
+  if (tid < 8) reinterpret_cast<uint32_t*>(smem + 768)[tid] = 0u;   // the zero B entry
+  __syncthreads();
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      const uint64_t pol = l2_evict_first_policy();
+      auto issue = [&](int t) {
+        const int u = t / KBR, br = t - u * KBR, slot = t % nslot;
+        const int nb = min(RB, KB - RB * br);
+        tag[slot] = t;   // before the arrive below, which releases it to the waiters
+        mbar_expect_tx(full + slot, (uint32_t)nb * 512u);
+        bulk_g2s_hint(ring + (size_t)slot * kMmaItemBytes, codes + (r_lo / 8 + u) * 4L * K + (long)br * RB * 512,
+                      (uint32_t)nb * 512u, full + slot, pol);
+      };
+      const bool stage_meta = meta_bytes > 0 && nrows > 0;
+      mbar_expect_tx(xbar, (uint32_t)K * 2u + (stage_meta ? (uint32_t)((mw.a1 - mw.a0) + (mw.b1 - mw.b0)) : 0u));
+      if (stage_meta) {
+        bulk_g2s(ms, meta + mw.a0, (uint32_t)(mw.a1 - mw.a0), xbar);
+        if (mw.b1 > mw.b0) bulk_g2s(ms + mw.bpl, meta + mw.b0, (uint32_t)(mw.b1 - mw.b0), xbar);
+      }
+      // a few weight runs before waiting for the previous kernel (weights do not
+      // depend on it); the activations are then queued ahead of the rest
+      int t = 0;
+      for (; t < nitems && t < nslot && t < kMmaPrefetch; ++t) issue(t);
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      bulk_g2s(smem + L.xraw, X, (uint32_t)K * 2u, xbar);
+      for (; t < nitems && t < nslot; ++t) issue(t);
+      for (; t < nitems; ++t) {
+        if (!mbar_wait(empty + t % nslot, (uint32_t)(t / nslot - 1) & 1u)) {
+          *abort_p = 1;
+          report(d_status, QNT_ERR_TIMEOUT);
+          break;
+        }
+        issue(t);
+      }
+      // drain: every issued copy has landed before the CTA exits
+      mbar_wait(xbar, 0);
+      for (int i = (t > nslot ? t - nslot : 0); i < t; ++i) mbar_wait(full + i % nslot, (uint32_t)(i / nslot) & 1u);
+    }
+  } else {
+    // ---------------------------------------------------------------- consumers
+    const int cw = warp - 1;
+    if (!mbar_wait(xbar, 0)) { *abort_p = 1; report(d_status, QNT_ERR_TIMEOUT); }
+    if (!*abort_p) {
+#pragma unroll 2
+      for (int b = cw; b < KB; b += kMmaConsumers) mma_build_x<FMT, G>(xraw_a, xf_a, xs2_a, b, xbf16, lane);
+    }
+    asm volatile("bar.sync 1, %0;" :: "n"(32 * kMmaConsumers) : "memory");
+
+    const int g = lane >> 2, r = lane & 3;                       // A: row g, chunk r
+    const int hB = lane >> 3, sB = (lane >> 2) & 1;              // B: column 2 hB + sB
+    const bool bload = hB < GPB && r / (4 / GPB) == hB;
+    const uint32_t xb_a = bload ? xf_a + 16u * (uint32_t)(4 * sB + r) : zero_a;
+    const uint32_t xstride = bload ? 256u : 0u, xhi = bload ? 128u : 16u;   // lanes without B read zeros
+    const uint32_t coff = 64u * g + 16u * (uint32_t)(r ^ ((g >> 1) & 3));
+    const int re = r < GPB ? r : GPB - 1;                        // epilogue group (lanes r < GPB)
+    const int ra = r / (4 / GPB);                                // group of this lane's chunk
+    // staged metadata: plane A (scales) and plane B (zeros / selectors) by group index
+    constexpr int PA = MetaPlanes<FMT>::A;
+    const uint32_t msa = smem_addr(ms) - (uint32_t)mw.a0;
+    const uint32_t msb = smem_addr(ms) + (uint32_t)(mw.bpl + z0 - mw.b0);
+    for (int t = cw; t < nitems && !*abort_p; t += kMmaConsumers) {
+      const int u = t / KBR, br = t - u * KBR, slot = t % nslot;
+      const long row = r_lo + 8 * u + g;
+      const bool rowok = row < r_hi;
+      const bool ok = rowok && r < GPB;
+      const long rowm = rowok ? row : r_lo;                      // a row whose metadata is staged
+      const int nb = min(RB, KB - RB * br);
+      const int b0 = RB * br;
+      const int f0 = (int)(rowm * GK) + b0 * GPB;                // group of block b0 in this lane's row
+      if (!rg_wait_item(tag, full, slot, t, nslot, abort_p)) { *abort_p = 1; report(d_status, QNT_ERR_TIMEOUT); break; }
+      const uint32_t ca = ring_a + (uint32_t)slot * kMmaItemBytes + coff;
+      float yacc = 0.0f;
+#pragma unroll 2
+      for (int bi = 0; bi < nb; ++bi) {
+        const int b = b0 + bi;
+        const uint4 cv = lds128a(ca + 512u * bi);
+        const uint4 x0 = lds128a(xb_a + xstride * b), x1 = lds128a(xb_a + xstride * b + xhi);
+        const float2 sc = lds64fa(xs2_a + 8u * (uint32_t)(b * GPB + re));   // (c / 2^e, group sum of x)
+        const int fe = f0 + bi * GPB + re, fa = f0 + bi * GPB + ra;
+        float ms_s, ms_t = 0.0f;                                   // this lane's epilogue metadata
+        uint32_t sv16 = 0;
+        if (meta_bytes > 0) {
+          if (FMT == QNT_FP4_AFPQ) {
+            const uint32_t v = lds32a(msa + 4u * fe);
+            ms_s = h2f(v & 0xFFFFu);
+            ms_t = h2f(v >> 16);
+          } else {
+            ms_s = h2f(lds16a(msa + 2u * fe));
+          }
+          if (FMT == QNT_INT4_ASYM) ms_t = (float)((lds8a(msb + (uint32_t)(fe >> 1)) >> (4 * (fe & 1))) & 15u);
+          if (FMT == QNT_FP4_RAZER) {
+            const uint32_t sel = (lds8a(msb + (uint32_t)(fa >> 2)) >> (2 * (fa & 3))) & 3u;
+            sv16 = ((sel & 2u) ? 0x4800u : 0x4500u) | ((sel & 1u) ? 0x8000u : 0u);   // +-8 or +-5
+          }
+        } else {
+          const GroupMeta md = group_meta<FMT>(meta, z0, fe);
+          ms_s = md.s;
+          ms_t = md.t;
+          if (FMT == QNT_INT4_ASYM) { ms_s *= 1.0f / 16777216.0f; ms_t = ms_s == 0.0f ? 0.0f : md.t / ms_s; }
+          if (FMT == QNT_FP4_RAZER) sv16 = __half_as_ushort(__float2half_rn(group_meta<FMT>(meta, z0, fa).t));
+        }
+        const uint32_t w[4] = {cv.x, cv.y, cv.z, cv.w};
+        const uint32_t bx[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        // two accumulator chains (MMAs 0, 2 and 1, 3)
+        float d[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+        float dn[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (FMT == QNT_INT4_ASYM) {
+            const uint32_t w8 = w[j] >> 8;
+            mma_16816(d[j & 1], w[j] & 0x000F000Fu, w8 & 0x000F000Fu, w[j] & 0x00F000F0u, w8 & 0x00F000F0u,
+                      bx[2 * j], bx[2 * j + 1]);
+          } else {
+            uint32_t h[4];
+            cvt_e2m1x8(w[j], h[0], h[1], h[2], h[3]);
+            if (FMT == QNT_FP4_RAZER) {
+              // codes 0b1000 (decoded as -0) take the group's special value
+              const uint32_t tt = (w[j] & 0x77777777u) + 0x77777777u;
+              const uint32_t spec = lop3<0x20>(w[j], tt, 0x88888888u);
+#pragma unroll
+              for (int pp = 0; pp < 4; ++pp) {
+                if (spec & (0x8u << (8 * pp))) h[pp] = (h[pp] & 0xFFFF0000u) | sv16;
+                if (spec & (0x80u << (8 * pp))) h[pp] = (h[pp] & 0x0000FFFFu) | (sv16 << 16);
+              }
+            }
+            if (FMT == QNT_FP4_AFPQ) {
+              uint32_t hp[4], hn[4];
+#pragma unroll
+              for (int pp = 0; pp < 4; ++pp) { hp[pp] = hmax2(h[pp], 0u); hn[pp] = hsub2(h[pp], hp[pp]); }
+              mma_16816(d[j & 1], hp[0], hp[1], hp[2], hp[3], bx[2 * j], bx[2 * j + 1]);
+              mma_16816(dn[j & 1], hn[0], hn[1], hn[2], hn[3], bx[2 * j], bx[2 * j + 1]);
+            } else {
+              mma_16816(d[j & 1], h[0], h[1], h[2], h[3], bx[2 * j], bx[2 * j + 1]);
+            }
+          }
+        }
+        const float v = (d[0][0] + d[0][3]) + (d[1][0] + d[1][3]);
+        float c;
+        if (FMT == QNT_INT4_ASYM) {
+          c = ms_s * (sc.x * v - ms_t * sc.y);
+        } else if (FMT == QNT_FP4_AFPQ) {
+          c = sc.x * (ms_s * v + ms_t * ((dn[0][0] + dn[0][3]) + (dn[1][0] + dn[1][3])));
+        } else {
+          c = ms_s * sc.x * v;
+        }
+        yacc += ok ? c : 0.0f;
+      }
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_addr(empty + slot)) : "memory");
+      if (GPB > 1) yacc += __shfl_xor_sync(0xffffffffu, yacc, 1);
+      if (GPB > 2) yacc += __shfl_xor_sync(0xffffffffu, yacc, 2);
+      if (r == 0 && rowok) part[(size_t)(8 * u + g) * KBR + br] = yacc;
+    }
+  }
+  __syncthreads();
+  for (int rl = tid; rl < nrows; rl += kMmaThreads) {
+    float v = 0.0f;
+    for (int br = 0; br < KBR; ++br) v += part[(size_t)rl * KBR + br];
+    if (xbf16) reinterpret_cast<__nv_bfloat16*>(Y)[r_lo + rl] = __float2bfloat16_rn(v);
+    else reinterpret_cast<__half*>(Y)[r_lo + rl] = __float2half_rn(v);
+  }
+}
+
 // ------------------------------------------------------------------ launchers
 int num_sms() {
   static int sms[64] = {0};
@@ -965,6 +1267,45 @@ static cudaError_t launch_rg(const qnt_desc& d, const void* codes, const void* m
                             d.N, d.K, xbf16, rows_cap, nslot, (int)mb, st);
 }
 
+template <int FMT, int G>
+static cudaError_t launch_mma(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
+                              int xbf16, int* st, cudaStream_t s, bool* handled) {
+  // two CTAs per SM where the shared memory allows it: the row groups are split
+  // over twice the SM count
+  const int NG = (d.N + 7) / 8;
+  const int grid = NG < 2 * num_sms() ? NG : 2 * num_sms();
+  const int rows_cap = 8 * ((NG + grid - 1) / grid);
+  auto total = [&](int ns, size_t mb) { return smem_mma_layout(d.K, G, rows_cap, ns, mb).total; };
+  size_t mb = meta_stage_bytes<FMT>(rows_cap, d.K / G);
+  int nslot = 0;
+  for (size_t cap : {(size_t)kMmaSmemCap, (size_t)kMaxDynSmem}) {
+    for (size_t m : {mb, (size_t)0}) {
+      for (int ns = kMmaMaxSlots; ns >= 2 && nslot == 0; --ns)
+        if (total(ns, m) <= cap) { nslot = ns; mb = m; }
+      if (nslot) break;
+    }
+    if (nslot) break;
+  }
+  if (nslot == 0) return cudaSuccess;   // not handled
+  const size_t smem = total(nslot, mb);
+  auto kfn = gemv4_mma_kernel<FMT, G>;
+  cudaError_t e = configure_smem(reinterpret_cast<const void*>(kfn));
+  if (e != cudaSuccess) return e;
+  *handled = true;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kMmaThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kfn, static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(meta), z0, X, Y,
+                            d.N, d.K, xbf16, rows_cap, nslot, (int)mb, st);
+}
+
 // One activation vector, 4-bit formats: the register-resident kernel above.
 // *handled = false when it does not take the shape.
 cudaError_t launch_gemv4_one(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
@@ -972,9 +1313,9 @@ cudaError_t launch_gemv4_one(const qnt_desc& d, const void* codes, const void* m
   *handled = false;
 #define QNT_RG(FMT)                                                                          \
   switch (d.group) {                                                                         \
-    case 32: return launch_rg<FMT, 32>(d, codes, meta, z0, X, Y, xbf16, st, s, handled);     \
-    case 64: return launch_rg<FMT, 64>(d, codes, meta, z0, X, Y, xbf16, st, s, handled);     \
-    default: return launch_rg<FMT, 128>(d, codes, meta, z0, X, Y, xbf16, st, s, handled);    \
+    case 32: return launch_mma<FMT, 32>(d, codes, meta, z0, X, Y, xbf16, st, s, handled);    \
+    case 64: return launch_mma<FMT, 64>(d, codes, meta, z0, X, Y, xbf16, st, s, handled);    \
+    default: return launch_mma<FMT, 128>(d, codes, meta, z0, X, Y, xbf16, st, s, handled);   \
   }
   switch (d.fmt) {
     case QNT_INT4_ASYM: QNT_RG(QNT_INT4_ASYM)

@@ -55,7 +55,7 @@ cudaError_t dispatch_gemm(const qnt_desc& d, const void* codes, const void* meta
   const long z0 = zero_plane(d);
   bool handled = false;
   cudaError_t e = cudaSuccess;
-  if (force == 0 && M == 1 && d.fmt != QNT_FP4_RAZER) {
+  if (force == 0 && M == 1) {
     e = qnt::launch_gemv4_one(d, codes, meta, z0, X, Y, xbf16, st, s, &handled);
     if (handled || e != cudaSuccess) return e;
   }

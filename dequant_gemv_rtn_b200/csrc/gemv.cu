@@ -821,10 +821,10 @@ gemv4_rg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ m
 // maximum in [2^14, 2^15); B entries of INT4 nibbles at bits 4..7 carry x / 16.
 constexpr int kMmaConsumers = 7;
 constexpr int kMmaThreads = 32 * (1 + kMmaConsumers);
-constexpr int kMmaRangeBlocks = 8;                        // blocks per work item
-constexpr int kMmaItemBytes = kMmaRangeBlocks * 512;      // 4 KB: one row group x 8 blocks
-constexpr int kMmaMaxSlots = 24;
-constexpr int kMmaPrefetch = 4;                           // items requested before the activations
+constexpr int kMmaRangeBlocks = 16;                       // blocks per work item
+constexpr int kMmaItemBytes = kMmaRangeBlocks * 512;      // 8 KB: one row group x 16 blocks
+constexpr int kMmaMaxSlots = 12;
+constexpr int kMmaPrefetch = 1;                           // items requested before the activations
 constexpr int kMmaCtrl = 1024;                            // barriers, tags, 32 zero bytes at 768
 constexpr int kMmaSmemCap = 113 * 1024;                   // two CTAs per SM
 

@@ -1,4 +1,5 @@
-// gemv.cu -- CUDA-core fused-dequant GEMV / multi-vector GEMV (all formats).
+// gemv.cu -- fused-dequant GEMV: the batch-1 tensor-core kernel for 4-bit
+// formats (mma.sync, below) and the CUDA-core multi-vector kernel (all formats).
 //
 // The decode-time kernel the RTN page ("Is (Selective) Round-To-Nearest
 // Quantization All You Need?", English abstract: token-generation throughput of
@@ -7,9 +8,9 @@
 // into FP16 with bit-level operations, fused with the dot product) describe:
 //   y[m][n] = sum_k dq(code[n][k], meta[n][k/g]) * x[m][k].
 //
-// This is the CUDA-core path: INT8 and FP16 weights, AFPQ, and batches too large
-// for the tensor-core kernel (gemv_tc.cu) take it.  One CTA of 16 warps per SM
-// owns a contiguous range of rows.
+// The CUDA-core multi-vector kernel: INT8 and FP16 weights, small batches of
+// FP4 / AFPQ, and batches too large for the tcgen05 kernel (gemv_tc.cu) take
+// it.  One CTA of 16 warps per SM owns a contiguous range of rows.
 //  * Activations are staged once per CTA with bulk copies; bf16 vectors are
 //    rescaled by an exact power of two into fp16 range.
 //  * A work item is (2 rows) x (2048 bytes of each row); each warp streams its
@@ -516,101 +517,23 @@ gemv_simt_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ 
   }
 }
 
-// ------------------------------------------------------------------ 4-bit kernel, one vector
-// Batch 1 keeps each lane's activations in registers.  Lane l owns block l
-// (128 weights) of a 32-block range of K: its 128 activations (64 registers),
-// and for INT4 its group sums, are loaded once per range.  A work item is one
-// row group (8 rows) x one range, a contiguous 16 KB run of the packed layout
-// fetched with one bulk copy into a CTA-wide ring by a producer warp.  In step
-// `it` of an item, lane l processes row (l + it) % 8 of the group: the eight
-// lanes of a shared-memory phase then read one chunk of eight different rows,
-// which the layout's chunk swizzle spreads over eight bank groups.  Per-row
-// partial sums are folded across lanes with shuffles and combined across
-// ranges in a fixed order.
-constexpr int kRgConsumers = 3;                           // 128-thread CTAs: two fit an SM
-constexpr int kRgThreads = 32 * (1 + kRgConsumers);
-constexpr int kRgLanesBlocks = 32;                        // blocks per range
-constexpr int kRgItemBytes = 8 * kRgLanesBlocks * 64;     // 16 KB
-constexpr int kRgMaxSlots = 8;
-constexpr int kRgCtrl = 1024;
-constexpr int kRgSmemCap = 113 * 1024;                    // leaves room for a second CTA
-
-struct SmemRg { size_t ring, xs, part, ms, total; };
-__host__ __device__ inline SmemRg smem_rg_layout(int K, int rows_cap, int nslot, size_t meta_bytes) {
-  const int KBR = (K / 128 + kRgLanesBlocks - 1) / kRgLanesBlocks;
-  SmemRg L;
-  L.ring = kRgCtrl;
-  L.xs = L.ring + (size_t)nslot * kRgItemBytes;
-  L.part = align16(L.xs + (size_t)K * 2);
-  L.ms = align16(L.part + (size_t)rows_cap * KBR * 4);
-  L.total = align16(L.ms + meta_bytes);
-  return L;
-}
-
-// x of this lane's block: 16 uint4 of fp16 (bf16 inputs scaled by 2^e into fp16
-// range, exactly; inv = 2^-e undoes it), INT4 group sums of the unscaled values.
-template <int FMT, int G>
-__device__ __forceinline__ void rg_load_x(const uint8_t* xs, long b, int KB, int xbf16, uint4 (&xr)[16],
-                                          float (&xgs)[128 / G], float& inv) {
-  constexpr int GPB = 128 / G;
-#pragma unroll
-  for (int q = 0; q < GPB; ++q) xgs[q] = 0.0f;
-  inv = 1.0f;
-  if (b >= KB) {
-#pragma unroll
-    for (int u = 0; u < 16; ++u) xr[u] = make_uint4(0, 0, 0, 0);
-    return;
-  }
-  const uint8_t* src = xs + b * 256;
-#pragma unroll
-  for (int u = 0; u < 16; ++u) xr[u] = lds128(src + 16 * u);
-  if (xbf16) {
-    float am = 0.0f;
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      const uint32_t w[4] = {xr[u].x, xr[u].y, xr[u].z, xr[u].w};
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        am = fmaxf(am, fabsf(__uint_as_float(w[p] << 16)));
-        am = fmaxf(am, fabsf(__uint_as_float(w[p] & 0xFFFF0000u)));
-      }
-    }
-    int e = 0;
-    if (am > 0.0f && isfinite(am)) e = min(max(14 - (int)((__float_as_uint(am) >> 23) & 255u) + 127, -126), 126);
-    const float f = __uint_as_float((uint32_t)(127 + e) << 23);
-    inv = __uint_as_float((uint32_t)(127 - e) << 23);
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      uint32_t w[4] = {xr[u].x, xr[u].y, xr[u].z, xr[u].w};
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const float lo = __uint_as_float(w[p] << 16), hi = __uint_as_float(w[p] & 0xFFFF0000u);
-        if (FMT == QNT_INT4_ASYM) xgs[(8 * u) / G] += lo + hi;
-        const __half2 h = __floats2half2_rn(lo * f, hi * f);
-        w[p] = *reinterpret_cast<const uint32_t*>(&h);
-      }
-      xr[u] = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-  } else if (FMT == QNT_INT4_ASYM) {
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      const uint32_t w[4] = {xr[u].x, xr[u].y, xr[u].z, xr[u].w};
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&w[p]));
-        xgs[(8 * u) / G] += f2.x + f2.y;
-      }
-    }
-  }
-}
-
-// Wait until ring slot `slot` holds item t and its bytes have landed.  The tag
+// ------------------------------------------------------------------ batch 1 on the tensor cores (mma.sync)
+// One activation vector, 4-bit formats.  A producer warp streams 8 KB runs of
+// the packed layout (one row group x 16 blocks of K, contiguous) into a
+// CTA-wide ring of slots with bulk copies; consumer warps take the runs in turn
+// and hand the multiply-adds to mma.sync m16n8k16 (fp16 inputs, fp32
+// accumulation) straight from the packed codes, so a lane spends five bit
+// operations and one MMA on eight weights.  Per-row partial sums of the runs are
+// combined in a fixed order (deterministic results).  Two CTAs per SM.
+//
+// Wait until ring slot `slot` holds item t and its bytes have landed, for
+// consumers that share one slot ring and each take every n-th item.  The tag
 // is read first: the producer writes t there only after the slot's previous
 // item has been consumed, so from then on the slot barrier's pending (or last
 // completed) phase is the one for t, and the parity wait cannot be met by a
 // phase two behind.  Bounded like every wait; false on timeout or abort.
-__device__ __forceinline__ bool rg_wait_item(volatile int* tag, uint64_t* full, int slot, int t, int nslot,
-                                             volatile int* abort_p) {
+__device__ __forceinline__ bool ring_wait_item(volatile int* tag, uint64_t* full, int slot, int t, int nslot,
+                                               volatile int* abort_p) {
   for (int it = 0; it < kMaxTries; ++it) {
     if (tag[slot] == t) {
       __threadfence_block();
@@ -622,191 +545,6 @@ __device__ __forceinline__ bool rg_wait_item(volatile int* tag, uint64_t* full, 
   return false;
 }
 
-template <int FMT, int G>
-__global__ void __launch_bounds__(kRgThreads, 1)
-gemv4_rg_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ meta, long z0,
-                const void* __restrict__ X, void* __restrict__ Y, int N, int K, int xbf16, int rows_cap,
-                int nslot, int meta_bytes, int* d_status) {
-  constexpr int GPB = 128 / G;              // groups per block
-  extern __shared__ __align__(1024) uint8_t smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
-  uint64_t* empty = full + kRgMaxSlots;
-  uint64_t* xbar = empty + kRgMaxSlots;
-  volatile int* abort_p = reinterpret_cast<volatile int*>(smem + 512);
-  // item last issued into each slot: consumers share the ring, so one may come
-  // to an item while its slot still holds an older one (see rg_wait_item)
-  volatile int* tag = reinterpret_cast<volatile int*>(smem + 640);
-  const SmemRg L = smem_rg_layout(K, rows_cap, nslot, (size_t)meta_bytes);
-  uint8_t* ring = smem + L.ring;
-  uint8_t* xs = smem + L.xs;
-  float* part = reinterpret_cast<float*>(smem + L.part);    // [rows_cap][KBR]
-  uint8_t* ms = smem + L.ms;
-  const int KB = K / 128, KBR = (KB + kRgLanesBlocks - 1) / kRgLanesBlocks, GK = K / G;
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  long r_lo, r_hi;
-  simt_rows(QNT_INT4_ASYM, N, blockIdx.x, gridDim.x, &r_lo, &r_hi);
-  const int nrows = (int)(r_hi - r_lo);
-  const int nitems = (nrows + 7) / 8 * KBR;
-  const MetaWin mw = meta_window<FMT>(r_lo, r_hi, GK, z0, rows_cap);
-
-  if (tid == 0) {
-    for (int i = 0; i < nslot; ++i) { mbar_init(full + i, 1); mbar_init(empty + i, 1); tag[i] = -1; }
-    mbar_init(xbar, 1);
-    *abort_p = 0;
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  }
-  __syncthreads();
-
-  if (warp == 0) {
-    // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      const uint64_t pol = l2_evict_first_policy();
-      auto issue = [&](int t) {
-        const int u = t / KBR, br = t - u * KBR, slot = t % nslot;
-        const int nb = min(kRgLanesBlocks, KB - kRgLanesBlocks * br);
-        tag[slot] = t;   // before the arrive below, which releases it to the waiters
-        mbar_expect_tx(full + slot, (uint32_t)nb * 512u);
-        bulk_g2s_hint(ring + (size_t)slot * kRgItemBytes, codes + (r_lo / 8 + u) * 4L * K + (long)br * kRgLanesBlocks * 512,
-                      (uint32_t)nb * 512u, full + slot, pol);
-      };
-      const bool stage_meta = meta_bytes > 0 && nrows > 0;
-      mbar_expect_tx(xbar, (uint32_t)K * 2u + (stage_meta ? (uint32_t)((mw.a1 - mw.a0) + (mw.b1 - mw.b0)) : 0u));
-      if (stage_meta) {
-        bulk_g2s(ms, meta + mw.a0, (uint32_t)(mw.a1 - mw.a0), xbar);
-        if (mw.b1 > mw.b0) bulk_g2s(ms + mw.bpl, meta + mw.b0, (uint32_t)(mw.b1 - mw.b0), xbar);
-      }
-      int t = 0;
-      for (; t < nitems && t < nslot; ++t) issue(t);   // weights do not depend on the previous kernel
-      asm volatile("griddepcontrol.wait;" ::: "memory");
-      bulk_g2s(xs, X, (uint32_t)K * 2u, xbar);
-      for (; t < nitems; ++t) {
-        if (!mbar_wait(empty + t % nslot, (uint32_t)(t / nslot - 1) & 1u)) {
-          *abort_p = 1;
-          report(d_status, QNT_ERR_TIMEOUT);
-          break;
-        }
-        issue(t);
-      }
-      // drain: every issued copy has landed before the CTA exits
-      mbar_wait(xbar, 0);
-      for (int i = (t > nslot ? t - nslot : 0); i < t; ++i) mbar_wait(full + i % nslot, (uint32_t)(i / nslot) & 1u);
-    }
-  } else {
-    // ---------------------------------------------------------------- consumers
-    const int cw = warp - 1;
-    if (!mbar_wait(xbar, 0)) { *abort_p = 1; report(d_status, QNT_ERR_TIMEOUT); }
-    uint4 xr[16];
-    float xgs[GPB];
-    float inv = 1.0f;
-    int cur_br = -1;
-    for (int t = cw; t < nitems && !*abort_p; t += kRgConsumers) {
-      const int u = t / KBR, br = t - u * KBR, slot = t % nslot;
-      const long b = (long)br * kRgLanesBlocks + lane;            // this lane's block
-      if (br != cur_br) { rg_load_x<FMT, G>(xs, b, KB, xbf16, xr, xgs, inv); cur_br = br; }
-      if (!rg_wait_item(tag, full, slot, t, nslot, abort_p)) { *abort_p = 1; report(d_status, QNT_ERR_TIMEOUT); break; }
-      const uint8_t* st = ring + (size_t)slot * kRgItemBytes + (size_t)lane * 512;
-      const bool has = b < KB;
-      float yit[8];
-#pragma unroll
-      for (int it = 0; it < 8; ++it) {
-        yit[it] = 0.0f;
-        const int i8 = (lane + it) & 7;
-        const long row = r_lo + 8 * u + i8;
-        if (!has || row >= r_hi) continue;
-#pragma unroll
-        for (int q = 0; q < GPB; ++q) {
-          const long f = row * GK + b * GPB + q;
-          const GroupMeta md = meta_bytes > 0 ? group_meta_s<FMT>(ms, mw, z0, f) : group_meta<FMT>(meta, z0, f);
-          float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-          const float corr = 0.0f;   // RaZeR special values are placed in the decoded operands
-          uint32_t sv16 = 0;
-          if (FMT == QNT_FP4_RAZER) sv16 = __half_as_ushort(__float2half_rn(md.t));   // +-5 or +-8, exact
-#pragma unroll
-          for (int cc = 0; cc < 4 / GPB; ++cc) {
-            const int c = q * (4 / GPB) + cc;                  // chunk of the block
-            const uint4 cv = lds128(st + 64 * i8 + 16 * (c ^ ((i8 >> 1) & 3)));
-            const uint32_t w[4] = {cv.x, cv.y, cv.z, cv.w};
-#pragma unroll
-            for (int jw = 0; jw < 4; ++jw) {
-              if (FMT == QNT_INT4_ASYM) {
-                // word jw: low nibbles -> chunk weights 4jw..4jw+3, high -> 16+4jw..16+4jw+3
-                const uint4 xa = xr[4 * c + jw / 2], xb = xr[4 * c + 2 + jw / 2];
-                const uint32_t xl0 = (jw & 1) ? xa.z : xa.x, xl1 = (jw & 1) ? xa.w : xa.y;
-                const uint32_t xh0 = (jw & 1) ? xb.z : xb.x, xh1 = (jw & 1) ? xb.w : xb.y;
-                const uint32_t w8 = w[jw] >> 8;
-                fma_mixed2(w[jw] & 0x000F000Fu, xl0, a[0], a[1]);
-                fma_mixed2(w8 & 0x000F000Fu, xl1, a[0], a[1]);
-                fma_mixed2(w[jw] & 0x00F000F0u, xh0, a[2], a[3]);
-                fma_mixed2(w8 & 0x00F000F0u, xh1, a[2], a[3]);
-              } else {
-                const uint4 x4 = xr[4 * c + jw];                // chunk weights 8jw..8jw+7
-                uint32_t h[4];
-                cvt_e2m1x8(w[jw], h[0], h[1], h[2], h[3]);
-                if (FMT == QNT_FP4_AFPQ) {
-#pragma unroll
-                  for (int pp = 0; pp < 4; ++pp) {
-                    const uint32_t vp = hmax2(h[pp], 0u);
-                    const uint32_t vn = hsub2(h[pp], vp);
-                    fma_mixed2(vp, (&x4.x)[pp], a[0], a[1]);
-                    fma_mixed2(vn, (&x4.x)[pp], a[2], a[3]);
-                  }
-                } else {
-                  if (FMT == QNT_FP4_RAZER) {
-                    // weights coded 0b1000 (decoded as -0) take the group's special
-                    // value: nibble 2pp / 2pp+1 is the low / high half of h[pp]
-                    const uint32_t tt = (w[jw] & 0x77777777u) + 0x77777777u;
-                    const uint32_t spec = lop3<0x20>(w[jw], tt, 0x88888888u);
-                    if (spec) {
-#pragma unroll
-                      for (int pp = 0; pp < 4; ++pp) {
-                        if (spec & (0x8u << (8 * pp))) h[pp] = (h[pp] & 0xFFFF0000u) | sv16;
-                        if (spec & (0x80u << (8 * pp))) h[pp] = (h[pp] & 0x0000FFFFu) | (sv16 << 16);
-                      }
-                    }
-                  }
-#pragma unroll
-                  for (int pp = 0; pp < 4; ++pp) fma_mixed2(h[pp], (&x4.x)[pp], a[0], a[1]);
-                }
-              }
-            }
-          }
-          float v = chunk_value<FMT>(md, a, corr);
-          if (FMT == QNT_INT4_ASYM) v = v * inv - md.t * xgs[q];
-          else v *= inv;
-          yit[it] += v;
-        }
-      }
-      __syncwarp();
-      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_addr(empty + slot)) : "memory");
-      // fold: lanes l, l+8, l+16, l+24 share rows; then lane r gathers row r
-      float tot = 0.0f;
-#pragma unroll
-      for (int it = 0; it < 8; ++it) {
-        float sv = yit[it];
-        sv += __shfl_xor_sync(0xffffffffu, sv, 8);
-        sv += __shfl_xor_sync(0xffffffffu, sv, 16);
-        tot += __shfl_sync(0xffffffffu, sv, (lane - it) & 7);   // lane (r - it) % 8 holds row r in step it
-      }
-      const long row = r_lo + 8 * u + lane;
-      if (lane < 8 && row < r_hi) part[(size_t)(8 * u + lane) * KBR + br] = tot;
-    }
-  }
-  __syncthreads();
-  for (int rl = tid; rl < nrows; rl += kRgThreads) {
-    float v = 0.0f;
-    for (int br = 0; br < KBR; ++br) v += part[(size_t)rl * KBR + br];
-    if (xbf16) reinterpret_cast<__nv_bfloat16*>(Y)[r_lo + rl] = __float2bfloat16_rn(v);
-    else reinterpret_cast<__half*>(Y)[r_lo + rl] = __float2half_rn(v);
-  }
-}
-
-// ------------------------------------------------------------------ batch 1 on the tensor cores (mma.sync)
-// The same producer ring as above, but the consumers hand the multiply-adds to
-// mma.sync m16n8k16 (fp16 inputs, fp32 accumulation) straight from the packed
-// layout, so a lane spends a handful of bit operations and one MMA on eight
-// weights instead of eight multiply-adds.
-//
 // One MMA covers the eight rows of a row group over 32 weights of each row.  Lane
 // t = 4g + r holds the 16-byte chunk r of row g of a block; word j of that chunk
 // feeds MMA j of the block.  A row g of the MMA's A operand is the row's first
@@ -856,50 +594,62 @@ __device__ __forceinline__ uint32_t xf_off(int b, int r, int s, int j, int hf) {
   return (uint32_t)(256 * b + 128 * (j >> 1) + 16 * (4 * s + r) + 8 * (j & 1) + 4 * hf);
 }
 
-// Activation image of block b, built by one warp: lane l takes x[128b + 4l ..
-// 4l + 3].  Within a chunk, the weight at offset o = 16 hf + 4j + 2s + e (INT4)
+// Activation image of blocks b0 and b1, built by one warp: lane l takes
+// x[128b + 4l .. 4l + 3] of each.  Within a chunk, the weight at offset o = 16 hf + 4j + 2s + e (INT4)
 // or 8j + 4hf + 2s + e (FP4 family) meets B half hf, segment s of MMA j.  Also
 // writes (c / 2^e, sum of x over group h) per (block, group) to xs2, c = 2^24
 // for INT4 (undoes the subnormal encoding), else 1.
 template <int FMT, int G>
-__device__ __forceinline__ void mma_build_x(uint32_t xraw, uint32_t xf, uint32_t xs2, int b, int xbf16, int lane) {
+__device__ __forceinline__ void mma_build_x(uint32_t xraw, uint32_t xf, uint32_t xs2, int b0, int b1, int xbf16,
+                                            int lane) {
+  // two blocks per call (b1 < 0: none), so their shuffle reductions overlap
   constexpr int GPB = 128 / G;
-  const uint2 raw = lds64a(xraw + 256 * b + 8 * lane);
-  float v[4];
-  if (xbf16) {
-    v[0] = __uint_as_float(raw.x << 16); v[1] = __uint_as_float(raw.x & 0xFFFF0000u);
-    v[2] = __uint_as_float(raw.y << 16); v[3] = __uint_as_float(raw.y & 0xFFFF0000u);
-  } else {
-    v[0] = h2f(raw.x & 0xFFFFu); v[1] = h2f(raw.x >> 16);
-    v[2] = h2f(raw.y & 0xFFFFu); v[3] = h2f(raw.y >> 16);
+  const int bb[2] = {b0, b1 >= 0 ? b1 : b0};
+  float v[2][4], am[2], sg[2];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const uint2 raw = lds64a(xraw + 256 * bb[q] + 8 * lane);
+    if (xbf16) {
+      v[q][0] = __uint_as_float(raw.x << 16); v[q][1] = __uint_as_float(raw.x & 0xFFFF0000u);
+      v[q][2] = __uint_as_float(raw.y << 16); v[q][3] = __uint_as_float(raw.y & 0xFFFF0000u);
+    } else {
+      v[q][0] = h2f(raw.x & 0xFFFFu); v[q][1] = h2f(raw.x >> 16);
+      v[q][2] = h2f(raw.y & 0xFFFFu); v[q][3] = h2f(raw.y >> 16);
+    }
+    am[q] = fmaxf(fmaxf(fabsf(v[q][0]), fabsf(v[q][1])), fmaxf(fabsf(v[q][2]), fabsf(v[q][3])));
+    sg[q] = (v[q][0] + v[q][1]) + (v[q][2] + v[q][3]);
   }
-  float am = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
-  float sgrp = (v[0] + v[1]) + (v[2] + v[3]);
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-    if (FMT == QNT_INT4_ASYM && o < G / 4) sgrp += __shfl_xor_sync(0xffffffffu, sgrp, o);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      am[q] = fmaxf(am[q], __shfl_xor_sync(0xffffffffu, am[q], o));
+      if (FMT == QNT_INT4_ASYM && o < G / 4) sg[q] += __shfl_xor_sync(0xffffffffu, sg[q], o);
+    }
   }
-  int e = 0;
-  if (am > 0.0f && isfinite(am)) e = min(max(14 - (int)((__float_as_uint(am) >> 23) & 255u) + 127, -126), 126);
-  const float f = __uint_as_float((uint32_t)(127 + e) << 23);
   const int r = lane >> 3, o = 4 * (lane & 7);
   int j, hf;
-  float fs = f;
   if (FMT == QNT_INT4_ASYM) {
     hf = o >> 4;
     j = (o & 15) >> 2;
-    if (hf) fs = f * 0.0625f;   // these weights decode 16x too large
   } else {
     j = o >> 3;
     hf = (o >> 2) & 1;
   }
-  const __half2 p0 = __floats2half2_rn(v[0] * fs, v[1] * fs), p1 = __floats2half2_rn(v[2] * fs, v[3] * fs);
-  sts32a(xf + xf_off(b, r, 0, j, hf), *reinterpret_cast<const uint32_t*>(&p0));
-  sts32a(xf + xf_off(b, r, 1, j, hf), *reinterpret_cast<const uint32_t*>(&p1));
-  if ((lane & (G / 4 - 1)) == 0) {
-    const float inv = __uint_as_float((uint32_t)(127 - e) << 23) * (FMT == QNT_INT4_ASYM ? 16777216.0f : 1.0f);
-    sts64fa(xs2 + 8 * (b * GPB + lane / (G / 4)), inv, FMT == QNT_INT4_ASYM ? sgrp : 0.0f);
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    if (q == 1 && b1 < 0) break;
+    int e = 0;
+    if (am[q] > 0.0f && isfinite(am[q])) e = min(max(14 - (int)((__float_as_uint(am[q]) >> 23) & 255u) + 127, -126), 126);
+    const float f = __uint_as_float((uint32_t)(127 + e) << 23);
+    const float fs = (FMT == QNT_INT4_ASYM && hf) ? f * 0.0625f : f;   // INT4 bits 4..7 decode 16x too large
+    const __half2 p0 = __floats2half2_rn(v[q][0] * fs, v[q][1] * fs), p1 = __floats2half2_rn(v[q][2] * fs, v[q][3] * fs);
+    sts32a(xf + xf_off(bb[q], r, 0, j, hf), *reinterpret_cast<const uint32_t*>(&p0));
+    sts32a(xf + xf_off(bb[q], r, 1, j, hf), *reinterpret_cast<const uint32_t*>(&p1));
+    if ((lane & (G / 4 - 1)) == 0)
+      sts64fa(xs2 + 8 * (bb[q] * GPB + lane / (G / 4)),
+              __uint_as_float((uint32_t)(127 - e) << 23) * (FMT == QNT_INT4_ASYM ? 16777216.0f : 1.0f),
+              FMT == QNT_INT4_ASYM ? sg[q] : 0.0f);
   }
 }
 
@@ -983,8 +733,8 @@ gemv4_mma_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ 
     const int cw = warp - 1;
     if (!mbar_wait(xbar, 0)) { *abort_p = 1; report(d_status, QNT_ERR_TIMEOUT); }
     if (!*abort_p) {
-#pragma unroll 2
-      for (int b = cw; b < KB; b += kMmaConsumers) mma_build_x<FMT, G>(xraw_a, xf_a, xs2_a, b, xbf16, lane);
+      for (int b = cw; b < KB; b += 2 * kMmaConsumers)
+        mma_build_x<FMT, G>(xraw_a, xf_a, xs2_a, b, b + kMmaConsumers < KB ? b + kMmaConsumers : -1, xbf16, lane);
     }
     asm volatile("bar.sync 1, %0;" :: "n"(32 * kMmaConsumers) : "memory");
 
@@ -1009,7 +759,7 @@ gemv4_mma_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ 
       const int nb = min(RB, KB - RB * br);
       const int b0 = RB * br;
       const int f0 = (int)(rowm * GK) + b0 * GPB;                // group of block b0 in this lane's row
-      if (!rg_wait_item(tag, full, slot, t, nslot, abort_p)) { *abort_p = 1; report(d_status, QNT_ERR_TIMEOUT); break; }
+      if (!ring_wait_item(tag, full, slot, t, nslot, abort_p)) { *abort_p = 1; report(d_status, QNT_ERR_TIMEOUT); break; }
       const uint32_t ca = ring_a + (uint32_t)slot * kMmaItemBytes + coff;
       float yacc = 0.0f;
 #pragma unroll 2
@@ -1226,48 +976,6 @@ int gemv_max_mb(const qnt_desc& d) {
 }
 
 template <int FMT, int G>
-static cudaError_t launch_rg(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
-                             int xbf16, int* st, cudaStream_t s, bool* handled) {
-  // two CTAs per SM: the row groups are split over twice the SM count, and a CTA
-  // small enough to share its SM lets the next kernel's CTAs start early
-  const int NG = (d.N + 7) / 8;
-  const int grid = NG < 2 * num_sms() ? NG : 2 * num_sms();
-  const int rows_cap = 8 * ((NG + grid - 1) / grid);
-  size_t mb = meta_stage_bytes<FMT>(rows_cap, d.K / d.group);
-  int nslot = kRgMaxSlots;
-  size_t cap = kRgSmemCap;
-  while (nslot > 2 && smem_rg_layout(d.K, rows_cap, nslot, mb).total > cap) --nslot;
-  if (smem_rg_layout(d.K, rows_cap, nslot, mb).total > cap) {   // alone on its SM, then
-    cap = kMaxDynSmem;
-    nslot = kRgMaxSlots;
-    while (nslot > 2 && smem_rg_layout(d.K, rows_cap, nslot, mb).total > cap) --nslot;
-  }
-  if (smem_rg_layout(d.K, rows_cap, nslot, mb).total > cap) {
-    mb = 0;   // metadata from global memory
-    nslot = kRgMaxSlots;
-    while (nslot > 2 && smem_rg_layout(d.K, rows_cap, nslot, 0).total > cap) --nslot;
-    if (smem_rg_layout(d.K, rows_cap, nslot, 0).total > cap) return cudaSuccess;   // not handled
-  }
-  const size_t smem = smem_rg_layout(d.K, rows_cap, nslot, mb).total;
-  auto kfn = gemv4_rg_kernel<FMT, G>;
-  cudaError_t e = configure_smem(reinterpret_cast<const void*>(kfn));
-  if (e != cudaSuccess) return e;
-  *handled = true;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kRgThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kfn, static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(meta), z0, X, Y,
-                            d.N, d.K, xbf16, rows_cap, nslot, (int)mb, st);
-}
-
-template <int FMT, int G>
 static cudaError_t launch_mma(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
                               int xbf16, int* st, cudaStream_t s, bool* handled) {
   // two CTAs per SM where the shared memory allows it: the row groups are split
@@ -1306,7 +1014,7 @@ static cudaError_t launch_mma(const qnt_desc& d, const void* codes, const void* 
                             d.N, d.K, xbf16, rows_cap, nslot, (int)mb, st);
 }
 
-// One activation vector, 4-bit formats: the register-resident kernel above.
+// One activation vector, 4-bit formats: the tensor-core kernel above.
 // *handled = false when it does not take the shape.
 cudaError_t launch_gemv4_one(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
                              int xbf16, int* st, cudaStream_t s, bool* handled) {

@@ -22,8 +22,10 @@ cudaError_t launch_quantize(const qnt_desc& d, const float* W, void* codes, void
 cudaError_t launch_gemv_simt(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X,
                              void* Y, int M, int xbf16, int* st, cudaStream_t s);
 
-// y = W x for one activation vector, 4-bit formats, on CUDA cores with the
-// activations in registers (gemv.cu).  *handled = false when it does not apply.
+// y = W x for one activation vector, 4-bit formats, on the tensor cores with
+// mma.sync straight from the packed codes (gemv.cu).  *handled = false when it
+// does not apply (the activation vector and a weight ring do not fit in shared
+// memory).
 cudaError_t launch_gemv4_one(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
                              int xbf16, int* st, cudaStream_t s, bool* handled);
 

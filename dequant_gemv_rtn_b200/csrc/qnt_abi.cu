@@ -37,9 +37,9 @@ int check(const qnt_desc* d) {
 
 // Y[m] = W x[m], m < M.  Kernel choice (measured on B200 with L2-cold weights,
 // 14336 x 4096 and the Llama-7B decode shapes):
-//   one vector, INT4 / FP4 / AFPQ   -> register-resident CUDA-core kernel
+//   one vector, 4-bit formats        -> batch-1 kernel (mma.sync tensor cores)
 //   INT4 2..8 vectors; FP4; AFPQ;
-//   RaZeR 1..2 vectors               -> CUDA-core multi-vector kernel
+//   RaZeR 2 vectors                  -> CUDA-core multi-vector kernel
 //   INT4 9..16, RaZeR 3..16 vectors  -> tensor-core kernel (tcgen05)
 //   INT8, FP16, more than 16 vectors -> CUDA-core multi-vector kernel
 // QNT_FORCE_SIMT=1 selects the CUDA-core multi-vector kernel everywhere and

@@ -51,9 +51,9 @@ def algo_bytes_int4(N, K, g=GROUP, M=1):
 STEP_BYTES = LAYERS * sum(algo_bytes_int4(N, K) for _, N, K in SHAPES)
 # DRAM bytes (read + write) per launch of the batch-1 INT4 kernel, averaged over
 # the five shapes of a layer, from single-launch cold-cache ncu captures
-# (profiles/gemv4_rg_int4_g128_decode_shapes.md).  Set to None whenever the
+# (profiles/gemv4_mma_int4_g128_decode_shapes.md).  Set to None whenever the
 # kernel changes until it is captured again.
-TRAFFIC_PER_LAUNCH = None
+TRAFFIC_PER_LAUNCH = 21094554
 
 
 def measured_peaks():

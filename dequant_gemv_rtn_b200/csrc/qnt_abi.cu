@@ -40,8 +40,9 @@ int check(const qnt_desc* d) {
 //   one vector, 4-bit formats        -> batch-1 kernel (mma.sync tensor cores)
 //   INT4 2..8 vectors; FP4; AFPQ;
 //   RaZeR 2 vectors                  -> CUDA-core multi-vector kernel
-//   INT4 9..16, RaZeR 3..16 vectors  -> tensor-core kernel (tcgen05)
-//   INT8, FP16, more than 16 vectors -> CUDA-core multi-vector kernel
+//   INT4 from 9, RaZeR from 3 vectors -> tensor-core kernel (tcgen05), in
+//                                       passes of 16 vectors above 16
+//   INT8, FP16; FP4 / AFPQ above 8    -> CUDA-core multi-vector kernel (passes of 8)
 // QNT_FORCE_SIMT=1 selects the CUDA-core multi-vector kernel everywhere and
 // QNT_FORCE_TC=1 the tensor-core kernel wherever it applies (used to test every
 // path on the same inputs).
@@ -60,11 +61,23 @@ cudaError_t dispatch_gemm(const qnt_desc& d, const void* codes, const void* meta
     if (handled || e != cudaSuccess) return e;
   }
   const bool tc = force == 2 || (force == 0 && ((d.fmt == QNT_INT4_ASYM && M > 8) || (d.fmt == QNT_FP4_RAZER && M > 2)));
+  int m0 = 0;   // vectors done
   if (tc) {
-    e = qnt::launch_gemv_tc(d, codes, meta, z0, X, Y, M, xbf16, st, s, &handled);
-    if (handled || e != cudaSuccess) return e;
+    // the tensor-core kernel takes up to 16 vectors per launch; larger batches
+    // run in passes of 16 (each pass streams the weights once)
+    while (m0 < M) {
+      const int mm = M - m0 < 16 ? M - m0 : 16;
+      handled = false;
+      e = qnt::launch_gemv_tc(d, codes, meta, z0, static_cast<const char*>(X) + (size_t)m0 * d.K * 2,
+                              static_cast<char*>(Y) + (size_t)m0 * d.N * 2, mm, xbf16, st, s, &handled);
+      if (e != cudaSuccess) return e;
+      if (!handled) break;
+      m0 += mm;
+    }
+    if (m0 == M) return cudaSuccess;
   }
-  return qnt::launch_gemv_simt(d, codes, meta, z0, X, Y, M, xbf16, st, s);
+  return qnt::launch_gemv_simt(d, codes, meta, z0, static_cast<const char*>(X) + (size_t)m0 * d.K * 2,
+                               static_cast<char*>(Y) + (size_t)m0 * d.N * 2, M - m0, xbf16, st, s);
 }
 
 }  // namespace

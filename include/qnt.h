@@ -122,7 +122,8 @@ typedef struct {
  *   QNT_FP4_E2M1 / AFPQ / RAZER:   8j + p
  * So 256 consecutive weights of eight rows are one contiguous 1 KB run (one
  * bulk copy), eight threads that read the same chunk of eight rows of a group
- * hit distinct shared-memory bank groups, and the INT4 order turns a word into
+ * (or the four chunks of two rows) hit distinct shared-memory bank groups, and
+ * the INT4 order turns a word into
  * fp16 pairs with two masks and one shift (low nibbles give chunk weights 0..15
  * in order, high nibbles 16..31).  FP4-family bytes hold two consecutive
  * weights, low nibble first.
@@ -169,8 +170,11 @@ int qnt_quantize(const qnt_desc* desc, const float* d_W, void* d_codes, void* d_
  *   d_x        device, [K] fp16 or bf16 (xdtype).
  *   d_y        device, [N] in the same type, written.
  *   d_status   device int or NULL: QNT_ERR_TIMEOUT if a staging wait expires.
- * Accuracy: |y - y_exact| <= 4e-3 * sum_k |dq(n,k) x[k]| per element (products
- * are exact in fp32, accumulation is fp32, one final rounding).  x is rescaled
+ * Accuracy: |y - y_exact| <= 4e-3 * sum_k |dq(n,k) x[k]| per element.  Every
+ * product is formed from exact fp16 operands and accumulated in fp32 (on the
+ * CUDA cores exactly; on the tensor cores, which take batch 1 and larger
+ * batches, within about 1e-4 of sum |products| as measured), with one final
+ * rounding to the output type.  x is rescaled
  * internally by a power of two so fp16 arithmetic cannot overflow.
  */
 int qnt_gemv(const qnt_desc* desc, const void* d_codes, const void* d_meta,

@@ -286,6 +286,7 @@ gemv_simt_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ 
                  const void* __restrict__ X, void* __restrict__ Y, int N, int K, int ldy, int xbf16,
                  int rows_cap, int meta_bytes, int* d_status) {
   constexpr bool Q4 = FMT != QNT_INT8_PERCHAN && FMT != QNT_FP16;
+  constexpr int Gd = G > 0 ? G : 1;                         // group size as a divisor (G = 0: INT8 / FP16)
   constexpr int WPC = FMT == QNT_INT8_PERCHAN ? 16 : 8;   // weights per 16-byte chunk (INT8 / FP16)
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* xbar = reinterpret_cast<uint64_t*>(smem);
@@ -402,15 +403,15 @@ gemv_simt_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ 
             const long k0 = (long)kr * kRange4 + 128 * h + 32 * c;   // first weight of the chunk
             GroupMeta md = {0.0f, 0.0f};
             if (row < r_hi)
-              md = meta_bytes > 0 ? group_meta_s<FMT>(ms, mw, z0, row * GK + k0 / G)
-                                  : group_meta<FMT>(meta, z0, row * GK + k0 / G);
+              md = meta_bytes > 0 ? group_meta_s<FMT>(ms, mw, z0, row * GK + k0 / Gd)
+                                  : group_meta<FMT>(meta, z0, row * GK + k0 / Gd);
 #pragma unroll
             for (int m = 0; m < MB; ++m) {
               float a[4] = {0.0f, 0.0f, 0.0f, 0.0f};
               float corr = 0.0f;
               dot_chunk4<FMT>(v, xs + (size_t)m * K + k0, a, corr);
               float val = chunk_value<FMT>(md, a, corr);
-              if (FMT == QNT_INT4_ASYM && (k0 % G) == 0) val -= md.t * xg[(size_t)m * GK + k0 / G];
+              if (FMT == QNT_INT4_ASYM && (k0 % Gd) == 0) val -= md.t * xg[(size_t)m * GK + k0 / Gd];
               acc[m] += val;
             }
           }
@@ -747,7 +748,6 @@ gemv4_mma_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ 
     const int re = r < GPB ? r : GPB - 1;                        // epilogue group (lanes r < GPB)
     const int ra = r / (4 / GPB);                                // group of this lane's chunk
     // staged metadata: plane A (scales) and plane B (zeros / selectors) by group index
-    constexpr int PA = MetaPlanes<FMT>::A;
     const uint32_t msa = smem_addr(ms) - (uint32_t)mw.a0;
     const uint32_t msb = smem_addr(ms) + (uint32_t)(mw.bpl + z0 - mw.b0);
     for (int t = cw; t < nitems && !*abort_p; t += kMmaConsumers) {

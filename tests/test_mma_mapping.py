@@ -1,0 +1,138 @@
+"""The batch-1 tensor-core GEMV's operand mapping, checked on the CPU.
+
+The kernel feeds mma.sync m16n8k16 straight from the packed codes: lane
+t = 4g + r holds chunk r of row g of a 128-weight block, word j of that chunk
+is MMA j's A fragment (row g: the word's first K segment, row g + 8: its
+second), and B column 2h + s holds segment s of the activations restricted to
+group h of the block.  This test restates that scheme (from the packed-layout
+text of include/qnt.h and the m16n8k16 fragment layout of the PTX ISA), runs
+the four MMAs of a block as fp64 matrix products and checks that
+D[g][2h] + D[g+8][2h+1], summed over the block's MMAs, is row g's dot product
+over group h.  A wrong mask, segment, activation position or fragment index
+fails it."""
+import numpy as np
+import pytest
+
+E2M1 = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def e2m1(c):
+    v = E2M1[c & 7]
+    return -v if c & 8 else v
+
+
+def nibble_weight(fmt, p, j):
+    """Chunk weight held by nibble p of word j (include/qnt.h, packed layout)."""
+    if fmt == "int4":
+        return 16 * (p % 2) + 4 * j + 2 * ((p // 2) % 2) + p // 4
+    return 8 * j + p
+
+
+def pack_block(fmt, q):
+    """q: [8 rows][128] codes of one block -> 512 bytes as 128 little-endian words."""
+    words = np.zeros(128, dtype=np.uint32)
+    for i in range(8):
+        for c in range(4):
+            pos = 4 * i + (c ^ ((i // 2) % 4))          # 16-byte chunk slot of row i, chunk c
+            for j in range(4):
+                w = 0
+                for p in range(8):
+                    w |= int(q[i, 32 * c + nibble_weight(fmt, p, j)]) << (4 * p)
+                words[4 * pos + j] = w
+    return words
+
+
+def half_pair(bits32):
+    lo, hi = bits32 & 0xFFFF, bits32 >> 16
+    return [float(np.array([lo], dtype=np.uint16).view(np.float16)[0]),
+            float(np.array([hi], dtype=np.uint16).view(np.float16)[0])]
+
+
+def a_fragments(fmt, w):
+    """The kernel's four A registers from one code word, as value pairs."""
+    if fmt == "int4":
+        w8 = w >> 8
+        regs = [w & 0x000F000F, w8 & 0x000F000F, w & 0x00F000F0, w8 & 0x00F000F0]
+        return [half_pair(r) for r in regs]     # fp16 subnormals q 2^-24 (16 q 2^-24 for bits 4..7)
+    # cvt.rn.f16x2.e2m1x2 of byte b: low nibble -> low half
+    return [[e2m1((w >> (8 * b)) & 15), e2m1((w >> (8 * b + 4)) & 15)] for b in range(4)]
+
+
+def b_entries(fmt, x, G):
+    """Activation image of one block: entry (s, r) = 4 MMAs x (b0, b1) value pairs.
+
+    Offset o of a chunk meets B half hf, segment s of MMA j where
+    o = 16 hf + 4j + 2s + e (INT4; half hf = 1 carries x / 16) or
+    o = 8j + 4hf + 2s + e (FP4 family)."""
+    ent = np.zeros((2, 4, 4, 2, 2))             # [s][r][j][hf][e]
+    for r in range(4):
+        for o in range(32):
+            e = o % 2
+            if fmt == "int4":
+                hf, j, s = o // 16, (o % 16) // 4, (o // 2) % 2
+                val = x[32 * r + o] / (16.0 if hf else 1.0)
+            else:
+                j, hf, s = o // 8, (o // 4) % 2, (o // 2) % 2
+                val = x[32 * r + o]
+            ent[s, r, j, hf, e] = val
+    return ent
+
+
+def emulate_block(fmt, q, x, G):
+    """Run the block's four MMAs with the kernel's lane assignments; return the
+    per-lane sums D[g][2r] + D[g+8][2r+1] (lane 4g + r)."""
+    GPB = 128 // G
+    words = pack_block(fmt, q)
+    ent = b_entries(fmt, x, G)
+    acc = np.zeros((16, 8))
+    for j in range(4):
+        A = np.zeros((16, 16))
+        B = np.zeros((16, 8))
+        for t in range(32):
+            g, r = t // 4, t % 4
+            # A: chunk r of row g, word j
+            w = int(words[4 * (4 * g + (r ^ ((g // 2) % 4))) + j])
+            a = a_fragments(fmt, w)
+            A[g, 2 * r:2 * r + 2] = a[0]
+            A[g + 8, 2 * r:2 * r + 2] = a[1]
+            A[g, 2 * r + 8:2 * r + 10] = a[2]
+            A[g + 8, 2 * r + 8:2 * r + 10] = a[3]
+            # B: column n = t / 4 = 2h + s; only lanes whose chunk r lies in group h load
+            n, hB, sB = t // 4, t // 8, (t // 4) % 2
+            if hB < GPB and r // (4 // GPB) == hB:
+                B[2 * r:2 * r + 2, n] = ent[sB, r, j, 0]
+                B[2 * r + 8:2 * r + 10, n] = ent[sB, r, j, 1]
+        acc += A @ B
+    return np.array([acc[t // 4, 2 * (t % 4)] + acc[t // 4 + 8, 2 * (t % 4) + 1] for t in range(32)])
+
+
+@pytest.mark.parametrize("fmt", ["int4", "fp4"])
+@pytest.mark.parametrize("G", [128, 64, 32])
+def test_block_mma_gives_row_group_dot_products(fmt, G):
+    rng = np.random.default_rng(G + (0 if fmt == "int4" else 1))
+    q = rng.integers(0, 16, size=(8, 128))
+    x = rng.standard_normal(128)
+    lanes = emulate_block(fmt, q, x, G)
+    GPB = 128 // G
+    scale = 2.0 ** -24 if fmt == "int4" else 1.0      # INT4 codes enter as fp16 subnormals
+    for g in range(8):
+        for h in range(4):
+            got = lanes[4 * g + h]
+            if h >= GPB:
+                assert got == 0.0                     # columns of absent groups stay zero
+                continue
+            ks = range(h * G, (h + 1) * G)
+            dq = [q[g, k] * scale if fmt == "int4" else e2m1(int(q[g, k])) for k in ks]
+            want = float(np.dot(dq, x[list(ks)]))
+            assert got == pytest.approx(want, rel=1e-12, abs=1e-30)
+
+
+def test_codes_reach_each_weight_once():
+    # every (row, weight) of a block enters exactly one A element of exactly one MMA
+    for fmt in ("int4", "fp4"):
+        seen = np.zeros((8, 128), dtype=int)
+        for c in range(4):
+            for j in range(4):
+                for p in range(8):
+                    seen[:, 32 * c + nibble_weight(fmt, p, j)] += 1
+        assert (seen == 1).all()

@@ -78,9 +78,24 @@ def b_entries(fmt, x, G):
     return ent
 
 
-def emulate_block(fmt, q, x, G):
+def razer_patch(w, pairs, sv):
+    """The kernel's RaZeR step: nibbles equal to 0b1000 (decoded -0), found with
+    t = (w & 0x77777777) + 0x77777777, spec = w & ~t & 0x88888888, take sv."""
+    t = ((w & 0x77777777) + 0x77777777) & 0xFFFFFFFF
+    spec = w & ~t & 0x88888888
+    out = [list(p) for p in pairs]
+    for b in range(4):
+        if spec & (0x8 << (8 * b)):
+            out[b][0] = sv
+        if spec & (0x80 << (8 * b)):
+            out[b][1] = sv
+    return out
+
+
+def emulate_block(fmt, q, x, G, sv=None, part=None):
     """Run the block's four MMAs with the kernel's lane assignments; return the
-    per-lane sums D[g][2r] + D[g+8][2r+1] (lane 4g + r)."""
+    per-lane sums D[g][2r] + D[g+8][2r+1] (lane 4g + r).  sv[g][h]: RaZeR special
+    value of row g, group h; part: AFPQ "pos" / "neg" operand (max(h, 0) / h - that)."""
     GPB = 128 // G
     words = pack_block(fmt, q)
     ent = b_entries(fmt, x, G)
@@ -93,6 +108,10 @@ def emulate_block(fmt, q, x, G):
             # A: chunk r of row g, word j
             w = int(words[4 * (4 * g + (r ^ ((g // 2) % 4))) + j])
             a = a_fragments(fmt, w)
+            if sv is not None:
+                a = razer_patch(w, a, sv[g][r // (4 // GPB)])   # the group of this lane's chunk
+            if part is not None:
+                a = [[max(v, 0.0) if part == "pos" else v - max(v, 0.0) for v in pr] for pr in a]
             A[g, 2 * r:2 * r + 2] = a[0]
             A[g + 8, 2 * r:2 * r + 2] = a[1]
             A[g, 2 * r + 8:2 * r + 10] = a[2]
@@ -136,3 +155,34 @@ def test_codes_reach_each_weight_once():
                 for p in range(8):
                     seen[:, 32 * c + nibble_weight(fmt, p, j)] += 1
         assert (seen == 1).all()
+
+
+@pytest.mark.parametrize("G", [128, 64, 32])
+def test_razer_special_values_follow_the_chunk_group(G):
+    rng = np.random.default_rng(100 + G)
+    q = rng.integers(0, 16, size=(8, 128))
+    q[:, ::5] = 8                                        # plenty of -0 codes in every group
+    x = rng.standard_normal(128)
+    GPB = 128 // G
+    sv = [[float(rng.choice([5.0, -5.0, 8.0, -8.0])) for _ in range(GPB)] for _ in range(8)]
+    lanes = emulate_block("razer", q, x, G, sv=sv)
+    for g in range(8):
+        for h in range(GPB):
+            ks = range(h * G, (h + 1) * G)
+            dq = [sv[g][h] if q[g, k] == 8 else e2m1(int(q[g, k])) for k in ks]
+            assert lanes[4 * g + h] == pytest.approx(float(np.dot(dq, x[list(ks)])), rel=1e-12)
+
+
+@pytest.mark.parametrize("G", [128, 32])
+def test_afpq_positive_and_negative_parts(G):
+    rng = np.random.default_rng(200 + G)
+    q = rng.integers(0, 16, size=(8, 128))
+    x = rng.standard_normal(128)
+    pos = emulate_block("afpq", q, x, G, part="pos")
+    neg = emulate_block("afpq", q, x, G, part="neg")
+    for g in range(8):
+        for h in range(128 // G):
+            ks = list(range(h * G, (h + 1) * G))
+            vals = np.array([e2m1(int(q[g, k])) for k in ks])
+            assert pos[4 * g + h] == pytest.approx(float(np.dot(np.maximum(vals, 0), x[ks])), rel=1e-12, abs=1e-15)
+            assert neg[4 * g + h] == pytest.approx(float(np.dot(np.minimum(vals, 0), x[ks])), rel=1e-12, abs=1e-15)

@@ -186,3 +186,27 @@ def test_afpq_positive_and_negative_parts(G):
             vals = np.array([e2m1(int(q[g, k])) for k in ks])
             assert pos[4 * g + h] == pytest.approx(float(np.dot(np.maximum(vals, 0), x[ks])), rel=1e-12, abs=1e-15)
             assert neg[4 * g + h] == pytest.approx(float(np.dot(np.minimum(vals, 0), x[ks])), rel=1e-12, abs=1e-15)
+
+
+def test_activation_image_offsets_agree_between_builder_and_reader():
+    """The builder stores the pair for (block b, chunk r, segment s, MMA j, half hf)
+    at byte 256 b + 128 (j >> 1) + 16 (4 s + r) + 8 (j & 1) + 4 hf; a lane reading
+    entry (s, r) loads 16 bytes at 256 b + 16 (4 s + r) and 16 at + 128, and takes
+    register 2 j + hf of the eight as MMA j's b0 (hf = 0) / b1 (hf = 1)."""
+    def written(b, r, s, j, hf):
+        return 256 * b + 128 * (j >> 1) + 16 * (4 * s + r) + 8 * (j & 1) + 4 * hf
+
+    def read(b, r, s, reg):
+        base = 256 * b + 16 * (4 * s + r) + (128 if reg >= 4 else 0)
+        return base + 4 * (reg % 4)
+
+    offsets = set()
+    for b in range(3):
+        for r in range(4):
+            for s in range(2):
+                for j in range(4):
+                    for hf in range(2):
+                        off = written(b, r, s, j, hf)
+                        assert off == read(b, r, s, 2 * j + hf)
+                        offsets.add(off)
+    assert sorted(offsets) == list(range(0, 3 * 256, 4))      # 256 bytes per block, no overlap

@@ -496,3 +496,152 @@ def test_nonfinite_weights_reported(orc):
     W[2, 5] = np.nan
     for fmt in (1, 2, 3, 4, 5, 6):
         assert orc.quantize(fmt, W, 128).status == orc.NONFINITE
+
+
+# ------------------------------------------------------------------ dequantization, by hand
+def _golden_e2m1_values():
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "e2m1_table.txt")) if l.strip() and not l.startswith("#")]
+    return {int(c): float(v) for c, v in rows}
+
+
+def _h(bits):
+    return float(np.uint16(bits).view(np.float16))
+
+
+# fp16 scales with many significant bits, distinct for s+ and s-
+_SP, _SN = 0x3A66, 0x2E1F
+
+
+def test_dequant_one_fp4_afpq_razer_int8_by_hand(orc):
+    """Each format's dequantized value from the golden E2M1 table (or the integer
+    code) times a chosen fp16 scale; AFPQ negative codes take s-, positive s+;
+    RaZeR's code 0b1000 decodes to the selected special value (+5, -5, +8, -8)."""
+    E = _golden_e2m1_values()
+    Sp, Sn = _h(_SP), _h(_SN)
+    assert Sp != Sn
+    for c in range(16):
+        assert orc.dequant_one(orc.FP4, c, _SP) == E[c] * Sp, c
+        want = E[c] * Sp if E[c] > 0 else E[c] * Sn
+        assert orc.dequant_one(orc.AFPQ, c, _SP, _SN) == want, c
+        for sel, sv in enumerate([5.0, -5.0, 8.0, -8.0]):
+            want = (sv if c == 8 else E[c]) * Sp
+            assert orc.dequant_one(orc.RAZER, c, _SP, 0, sel) == want, (c, sel)
+        for z in (0, 7, 15):
+            assert orc.dequant_one(orc.INT4, c, _SP, 0, z) == (c - z) * Sp, (c, z)
+    for q in (-127, -1, 0, 1, 77, 127):
+        assert orc.dequant_one(orc.INT8, q & 0xFF, _SN) == q * Sn, q
+
+
+@pytest.mark.parametrize("fmt", [1, 2, 3, 4, 5])
+def test_dequant_matrix_by_hand(orc, fmt):
+    """Whole-matrix dequantization with a different scale (and zero / selector)
+    for every group, or every row for INT8, against numpy arithmetic on the
+    golden E2M1 table: catches a wrong group or row index."""
+    rng = np.random.default_rng(40 + fmt)
+    N, K, g = 3, 256, 64
+    G = 1 if fmt == orc.INT8 else K // g
+    E = np.array([_golden_e2m1_values()[c] for c in range(16)])
+    s1 = rng.integers(0x2000, 0x3C00, size=N * G).astype(np.uint16)
+    s2 = rng.integers(0x2000, 0x3C00, size=N * G).astype(np.uint16)
+    z = rng.integers(0, 16 if fmt == orc.INT4 else 4, size=N * G).astype(np.uint8)
+    if fmt == orc.INT8:
+        codes = rng.integers(-127, 128, size=(N, K)).astype(np.int8).view(np.uint8)
+    else:
+        codes = rng.integers(0, 16, size=(N, K)).astype(np.uint8)
+    q = orc.Quant(fmt, N, K, K if fmt == orc.INT8 else g, codes, s1, s2 if fmt == orc.AFPQ else None,
+                  z if fmt in (orc.INT4, orc.RAZER) else None)
+    S1 = s1.view(np.float16).astype(np.float64).reshape(N, G)
+    S2 = s2.view(np.float16).astype(np.float64).reshape(N, G)
+    col = (np.arange(K) // g) if fmt != orc.INT8 else np.zeros(K, int)
+    S1k, S2k, Zk = S1[:, col], S2[:, col], z.reshape(N, G)[:, col].astype(np.float64)
+    if fmt == orc.INT4:
+        want = (codes - Zk) * S1k
+    elif fmt == orc.FP4:
+        want = E[codes] * S1k
+    elif fmt == orc.AFPQ:
+        v = E[codes]
+        want = np.where(v > 0, v * S1k, v * S2k)
+    elif fmt == orc.RAZER:
+        sv = np.array([5.0, -5.0, 8.0, -8.0])[z.reshape(N, G)[:, col]]
+        want = np.where(codes == 8, sv, E[codes]) * S1k
+    else:
+        want = codes.view(np.int8).astype(np.float64) * S1k
+    assert np.array_equal(orc.dequant(q), want)
+
+
+# ------------------------------------------------------------------ exact ties (hand-worked)
+def _tie_cases():
+    for line in open(os.path.join(GOLDEN, "int_ties.txt")):
+        if not line.strip() or line.startswith("#"):
+            continue
+        f = line.split()
+        name, fmt, log2s = f[0], f[1], int(f[2])
+        w = np.array([float(v) for v in f[3:11]]) * 2.0 ** log2s
+        yield name, fmt, w.astype(np.float32), int(f[11], 16), int(f[12]), [int(v) for v in f[13:21]]
+
+
+def test_int_ties_round_half_to_even(orc):
+    """INT4 codes and zero points and INT8 codes at exact .5 ties go to the even
+    integer (hand-worked groups in tests/golden/int_ties.txt)."""
+    cases = list(_tie_cases())
+    assert len(cases) == 3
+    for name, fmt, w, sbits, zero, codes in cases:
+        if fmt == "int4":
+            c, s1, _, z, st = orc.quantize_group(orc.INT4, w)
+            assert st == 0 and s1 == sbits and z == zero, name
+            assert list(c) == codes, (name, list(c))
+        else:
+            r = orc.quantize(orc.INT8, w[None, :], w.size)
+            assert r.status == 0 and int(r.s1[0]) == sbits, name
+            assert list(r.codes.view(np.int8)[0]) == codes, (name, list(r.codes.view(np.int8)[0]))
+
+
+# ------------------------------------------------------------------ RaZeR: summation order of the error
+def _razer_sq_errors(w, sel):
+    """Squared errors (binary64) of each weight under RaZeR candidate `sel`,
+    codes found by enumerating the whole grid (ties: regular value over the
+    special value, then even mantissa)."""
+    sv = [5.0, -5.0, 8.0, -8.0][sel]
+    am = np.float32(np.max(np.abs(w)))
+    s = float(np.float16(am / np.float32(max(6.0, abs(sv)))))
+    s = 1.0 if s == 0.0 else s
+    out = []
+    for x in w:
+        v = float(np.float32(x) / np.float32(s))
+        grid = [(abs(v - (sv if c == 8 else _e2m1_from_bits(c))), c == 8, c % 2, c) for c in range(16)]
+        d = min(t[0] for t in grid)
+        ties = [t for t in grid if t[0] == d]
+        reg = [t for t in ties if not t[1]]
+        c = (min(reg, key=lambda t: t[2])[3] if reg else 8)
+        e = float(x) - (sv if c == 8 else _e2m1_from_bits(c)) * s
+        out.append(e * e)
+    return out
+
+
+def _tree(t):
+    t, width = list(t), 1
+    while width < len(t):
+        for i in range(0, len(t) - width, 2 * width):
+            t[i] = t[i] + t[i + width]
+        width *= 2
+    return t[0]
+
+
+def test_razer_selector_uses_tree_order_sum(orc):
+    """A group whose candidates +5 and -5 tie under the balanced-tree sum of the
+    squared errors but not under a left-to-right sum: the selector is 0 (tree
+    tie, smallest selector), not 1 (tests/golden/razer_order_case.txt)."""
+    line = [l for l in open(os.path.join(GOLDEN, "razer_order_case.txt")) if l.strip() and not l.startswith("#")][0]
+    w = np.array([int(v, 16) for v in line.split()], np.uint32).view(np.float32)
+    E = [_razer_sq_errors(w, s) for s in range(4)]
+    tree = [_tree(e) for e in E]
+    seq = []
+    for e in E:                                    # plain left-to-right binary64 sum
+        acc = 0.0
+        for v in e:
+            acc += v
+        seq.append(acc)
+    assert tree[0] == tree[1] < min(tree[2], tree[3])
+    assert seq[1] < seq[0]                         # the case discriminates the two orders
+    codes, s1, _, sel, st = orc.quantize_group(orc.RAZER, w)
+    assert st == 0 and sel == 0

@@ -5,15 +5,21 @@ Workload (one "step" = one decode token through the stack's linear layers):
   32 layers x {qkv 4096->12288, o 4096->4096, gate 4096->11008, up 4096->11008,
   down 11008->4096}, INT4 asymmetric RTN, group 128, batch 1, fp16 activations
   x ~ N(0, 1), weights W = 0.02 * t5 * lognormal_row(0, 0.5) drawn on the GPU
-  with a seeded generator and quantized by qnt_quantize.  160 qnt_gemv calls per
-  step, 3.37 GB of packed weights per step: larger than L2, so every step reads
-  its weights from HBM (no flush needed).
+  with a seeded generator and quantized by qnt_quantize.  160 GEMVs per step,
+  3.37 GB of packed weights per step: larger than L2, so every step reads its
+  weights from HBM (no flush needed).
+
+The step is one qnt_gemv_seq call (one persistent kernel for the 160 GEMVs);
+every GEMV is marked `wait`, so it reads its x only after the previous GEMV of
+the step has written its y, as if x were computed from it.  Also reported: the
+same 160 GEMVs as separate qnt_gemv launches (programmatic dependent launch,
+captured in a CUDA graph), and each layer shape alone.
 
 Metric: achieved HBM GB/s from algorithmic bytes (codes + metadata + x + y per
-GEMV) and microseconds per decode layer (step time / 32).  The step's kernels
-are captured once in a CUDA graph and replayed; timing uses CUDA events on the
-launching stream, with a barrier and synchronize around the timed region and
-the max over ranks for N > 1 (each rank runs its own replica: weak scaling).
+GEMV) and microseconds per decode layer (step time / 32).  Timing uses CUDA
+events on the launching stream, with a barrier and synchronize around the timed
+region and the max over ranks for N > 1 (each rank runs its own replica: weak
+scaling).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 """
@@ -49,11 +55,9 @@ def algo_bytes_int4(N, K, g=GROUP, M=1):
 
 
 STEP_BYTES = LAYERS * sum(algo_bytes_int4(N, K) for _, N, K in SHAPES)
-# DRAM bytes (read + write) per launch of the batch-1 INT4 kernel, averaged over
-# the five shapes of a layer, from single-launch cold-cache ncu captures
-# (profiles/gemv4_mma_int4_g128_decode_shapes.md).  Set to None whenever the
-# kernel changes until it is captured again.
-TRAFFIC_PER_LAUNCH = 21094554
+# DRAM bytes (read + write) of one launch of the sequence kernel over the whole
+# stack, from an ncu capture of its current build (None: not captured yet).
+TRAFFIC_PER_LAUNCH = None
 
 
 def measured_peaks():
@@ -184,25 +188,60 @@ def run_ours(args, world, rank, local):
     ys = {(name, l): torch.empty(N, dtype=torch.float16, device="cuda")
           for l in range(LAYERS) for name, N, _ in SHAPES}
     stream = torch.cuda.Stream()
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    # decode-layer dependencies: each GEMV reads its x after the GEMV that
+    # produces it (o <- qkv, gate <- o, up <- o, down <- up and gate, the next
+    # layer's qkv <- down); as steps back in the sequence:
+    layer_wait = {"qkv": 1, "o": 1, "gate": 1, "up": 2, "down": 1}
+
+    def seq_items(x_of, y_of, waits=None):
+        return [(d, codes, meta, x_of(l, name, d), y_of(l, name),
+                 (waits or layer_wait)[name] if (l, name) != (0, "qkv") else 0)
+                for l, mods in enumerate(layers) for name, d, codes, meta in mods]
+
+    steps = Q.seq_steps(seq_items(lambda l, name, d: xs[d.K], lambda l, name: ys[(name, l)]))
+    serial = Q.seq_steps(seq_items(lambda l, name, d: xs[d.K], lambda l, name: ys[(name, l)],
+                                   {n: 1 for n in layer_wait}))
+    work = torch.zeros(Q.qnt_gemv_seq_work_bytes(len(steps)), dtype=torch.uint8, device="cuda")
+
+    def step_seq(s):
+        Q.qnt_gemv_seq(steps, Q.QNT_F16, work, st, s)
+
+    def step_serial(s):
+        Q.qnt_gemv_seq(serial, Q.QNT_F16, work, st, s)
 
     def step_launches(s):
         for l, mods in enumerate(layers):
             for name, d, codes, meta in mods:
-                Q.qnt_gemv(d, codes, meta, xs[d.K], ys[(name, l)], Q.QNT_F16, None, s)
+                Q.qnt_gemv(d, codes, meta, xs[d.K], ys[(name, l)], Q.QNT_F16, st, s)
 
-    # eager warm-up (also initializes per-kernel attributes before capture)
-    with torch.cuda.stream(stream):
-        step_launches(stream)
-    torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        step_launches(torch.cuda.current_stream())
-    torch.cuda.synchronize()
+    graphs = []   # every captured graph lives until the end of the run
 
-    for _ in range(args.warmup):
-        graph.replay()
-    torch.cuda.synchronize()
+    def time_graph(run, reps):
+        with torch.cuda.stream(stream):
+            run(stream)               # eager first (per-kernel attributes are set outside capture)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            run(torch.cuda.current_stream())
+        graphs.append(g)
+        for _ in range(args.warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        per = []
+        with torch.cuda.stream(stream):
+            for _ in range(reps):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                g.replay()
+                e1.record(stream)
+                per.append((e0, e1))
+        torch.cuda.synchronize()
+        return g, [x.elapsed_time(y) for x, y in per]
 
+    # headline: the sequence kernel, one launch per step
+    graph, _ = time_graph(step_seq, 1)
     sampler = ClockSampler(dev_index)
     sampler.start()
     time.sleep(0.3)
@@ -222,29 +261,27 @@ def run_ours(args, world, rank, local):
     ms = e0.elapsed_time(e1)
     ms = allreduce_max(ms, world)
     clocks = sampler.summary(t0, t1)
+    assert int(st.item()) == 0, f"device status {int(st.item())}"
+    # per-step distribution (separately timed replays)
+    _, seq_ms = time_graph(step_seq, max(10, min(args.steps, 200)))
+    # every GEMV waiting for the one before it
+    _, serial_ms = time_graph(step_serial, max(10, min(args.steps, 100)))
+    # the same GEMVs as separate launches (qnt_gemv, programmatic dependent launch)
+    _, chain_ms = time_graph(step_launches, max(10, min(args.steps, 100)))
 
+    pct = lambda v, q: float(np.percentile(v, q))
     # per-shape isolated launch times (same kernel, 32 cold layers per graph)
     per_shape = {}
     for mi, (name, N, K) in enumerate(SHAPES):
-        g2 = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g2, stream=stream):
+        def shape_launches(s, mi=mi, name=name, K=K):
             for l in range(LAYERS):
                 _, d, codes, meta = layers[l][mi]
-                Q.qnt_gemv(d, codes, meta, xs[K], ys[(name, l)], Q.QNT_F16, None, torch.cuda.current_stream())
-        for _ in range(3):
-            g2.replay()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        reps = 20
-        with torch.cuda.stream(stream):
-            a.record(stream)
-            for _ in range(reps):
-                g2.replay()
-            b.record(stream)
-        torch.cuda.synchronize()
-        us = a.elapsed_time(b) * 1000.0 / (reps * LAYERS)
-        per_shape[f"{name}_{K}x{N}"] = {"us": round(us, 3), "GBps": round(algo_bytes_int4(N, K) / us / 1e3, 1)}
-        del g2
+                Q.qnt_gemv(d, codes, meta, xs[K], ys[(name, l)], Q.QNT_F16, st, s)
+        _, shape_ms = time_graph(shape_launches, 20)
+        us = statistics.median(shape_ms) * 1000.0 / LAYERS
+        per_shape[f"{name}_{K}x{N}"] = {"us": round(us, 3), "GBps": round(algo_bytes_int4(N, K) / us / 1e3, 1),
+                                        "p10_p90_us": [round(pct(shape_ms, 10) * 1000.0 / LAYERS, 3),
+                                                       round(pct(shape_ms, 90) * 1000.0 / LAYERS, 3)]}
 
     # end to end through the public API with host buffers: per step, the step's
     # inputs (every GEMV's x, one pinned host buffer) go host->device in one copy
@@ -261,12 +298,12 @@ def run_ours(args, world, rank, local):
     d_out = torch.empty(ny, dtype=torch.float16, device="cuda")
     h_out = torch.empty(ny, dtype=torch.float16).pin_memory()
 
+    e2e_steps_desc = Q.seq_steps(seq_items(lambda l, name, d: d_in[x_off[(name, l)][0]:x_off[(name, l)][0] + d.K],
+                                           lambda l, name: d_out[y_off[(name, l)][0]:y_off[(name, l)][0] + y_off[(name, l)][1]]))
+
     def e2e_step(s):
         d_in.copy_(h_in, non_blocking=True)
-        for l, mods in enumerate(layers):
-            for name, d, codes, meta in mods:
-                (xo, K), (yo, N) = x_off[(name, l)], y_off[(name, l)]
-                Q.qnt_gemv(d, codes, meta, d_in[xo:xo + K], d_out[yo:yo + N], Q.QNT_F16, None, s)
+        Q.qnt_gemv_seq(e2e_steps_desc, Q.QNT_F16, work, st, s)
         h_out.copy_(d_out, non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -290,12 +327,13 @@ def run_ours(args, world, rank, local):
     e2e_ms = allreduce_max(a.elapsed_time(b), world) / e2e_steps
     h2d = LAYERS * sum(2 * K for _, _, K in SHAPES)
     d2h = LAYERS * sum(2 * N for _, N, _ in SHAPES)
-    del ge, graph
+    del ge
+    torch.cuda.synchronize()
+    graphs.clear()
 
     step_ms = ms / args.steps
     value = replica_value(STEP_BYTES, world, step_ms)
     peak, peak_kind = measured_peaks()
-    launches = LAYERS * len(SHAPES)
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(step_ms, 5), "higher_is_better": True, "scaling": "weak",
@@ -303,22 +341,34 @@ def run_ours(args, world, rank, local):
         "config": {"workload": WORKLOAD, "layers": LAYERS, "shapes_NxK": [[N, K] for _, N, K in SHAPES],
                    "group": GROUP, "batch": 1, "bytes_per_step": STEP_BYTES,
                    "l2": "inputs larger than L2 (3.37 GB of packed weights per step), no flush",
-                   "timing": "CUDA graph of one step replayed; CUDA events on the launching stream",
+                   "timing": "CUDA graph of one step (one qnt_gemv_seq call) replayed; CUDA events on the "
+                             "launching stream",
+                   "dependencies": "decode-layer order: each GEMV reads its x after the GEMV that produces it "
+                                   "(o<-qkv, gate<-o, up<-o, down<-gate,up, next qkv<-down)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "us_per_layer": round(step_ms * 1000.0 / LAYERS, 3),
-        "roofline": {"bound": "hbm", "achieved": round(STEP_BYTES / launches / (step_ms * 1e-3 / launches) / 1e9, 1),
+        "us_per_layer_p10_p90": [round(pct(seq_ms, 10) * 1000.0 / LAYERS, 3),
+                                 round(pct(seq_ms, 90) * 1000.0 / LAYERS, 3)],
+        "roofline": {"bound": "hbm", "achieved": round(STEP_BYTES / (step_ms * 1e-3) / 1e9, 1),
                      "peak": peak, "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy)" if peak_kind == "measured" else "fallback",
                      "unit": "GB/s", "frac": round(STEP_BYTES / (step_ms * 1e-3) / 1e9 / peak, 4),
-                     "traffic": TRAFFIC_PER_LAUNCH, "kernel": "gemv4_mma_kernel<INT4,g128>",
-                     "per_launch_bytes": STEP_BYTES // launches},
+                     "traffic": TRAFFIC_PER_LAUNCH, "kernel": "gemv1_kernel<INT4,g128> (sequence of 160 GEMVs)",
+                     "per_launch_bytes": STEP_BYTES, "launches_per_step": 1},
+        "serialized": {"us_per_layer": round(statistics.median(serial_ms) * 1000.0 / LAYERS, 3),
+                       "GBps": round(STEP_BYTES / (statistics.median(serial_ms) * 1e-3) / 1e9, 1),
+                       "how": "qnt_gemv_seq with every GEMV waiting for the one before it; median of replays"},
+        "per_launch_chain": {"us_per_layer": round(statistics.median(chain_ms) * 1000.0 / LAYERS, 3),
+                             "GBps": round(STEP_BYTES / (statistics.median(chain_ms) * 1e-3) / 1e9, 1),
+                             "how": "the same 160 GEMVs as qnt_gemv launches (programmatic dependent launch) "
+                                    "in one CUDA graph; median of replays"},
         "per_shape_isolated": per_shape,
-        "gpu_launches": launches * args.steps,
+        "gpu_launches": args.steps,
         "clocks": clocks,
         "e2e": {"value": round(replica_value(STEP_BYTES, world, e2e_ms), 1), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "how": "public C-ABI qnt_gemv per module; per step, every GEMV's x copied host->device from one "
-                       "pinned buffer and every y copied back in one device->host copy, inside a captured "
-                       "CUDA graph; weights resident"},
+                "how": "public C-ABI qnt_gemv_seq; per step, every GEMV's x copied host->device from one pinned "
+                       "buffer and every y copied back in one device->host copy, inside a captured CUDA graph; "
+                       "weights resident"},
     }
     return result, layers
 
@@ -393,32 +443,45 @@ def run_reference(args, world, rank, local):
 
 
 def run_kernel_only(name: str, fmt_name: str, repeats: int = 5):
-    """Small case for profilers: one matrix of the named decode shape, quantized
-    once, then `repeats` qnt_gemv launches (M=1, fp16 x)."""
+    """Small case for profilers.  A layer shape: one matrix of that shape,
+    quantized once, then `repeats` qnt_gemv launches (M=1, fp16 x).  "layer":
+    one decode layer (its five GEMVs) as `repeats` qnt_gemv_seq launches."""
     import torch
     from dequant_gemv_rtn_b200 import qnt as Q
     from dequant_gemv_rtn_b200 import synth
-    N, K = {n: (N, K) for n, N, K in SHAPES}[name]
     fmt = Q.FORMATS[fmt_name]
-    d = Q.desc(fmt, N, K, GROUP)
-    W = synth.llama_like_device(N, K, seed=3)
-    codes = torch.empty(Q.qnt_codes_bytes(d), dtype=torch.uint8, device="cuda")
-    meta = torch.empty(max(16, Q.qnt_meta_bytes(d)), dtype=torch.uint8, device="cuda")
-    Q.qnt_quantize(d, W, codes, meta)
-    del W
-    x = synth.activations_device(1, K, seed=5, dtype=torch.float16)
-    y = torch.empty(N, dtype=torch.float16, device="cuda")
-    for _ in range(repeats):
-        Q.qnt_gemv(d, codes, meta, x, y, Q.QNT_F16)
+    mats = []
+    for i, (n, N, K) in enumerate(SHAPES):
+        if name not in ("layer", n):
+            continue
+        d = Q.desc(fmt, N, K, GROUP)
+        W = synth.llama_like_device(N, K, seed=3 + i)
+        codes = torch.empty(Q.qnt_codes_bytes(d), dtype=torch.uint8, device="cuda")
+        meta = torch.empty(max(16, Q.qnt_meta_bytes(d)), dtype=torch.uint8, device="cuda")
+        Q.qnt_quantize(d, W, codes, meta)
+        del W
+        x = synth.activations_device(1, K, seed=5, dtype=torch.float16)
+        y = torch.empty(N, dtype=torch.float16, device="cuda")
+        mats.append((d, codes, meta, x, y))
+    if name == "layer":
+        steps = Q.seq_steps([(d, c, m, x, y, 1 if i else 0) for i, (d, c, m, x, y) in enumerate(mats)])
+        work = torch.zeros(Q.qnt_gemv_seq_work_bytes(len(steps)), dtype=torch.uint8, device="cuda")
+        for _ in range(repeats):
+            Q.qnt_gemv_seq(steps, Q.QNT_F16, work)
+    else:
+        d, codes, meta, x, y = mats[0]
+        for _ in range(repeats):
+            Q.qnt_gemv(d, codes, meta, x, y, Q.QNT_F16)
     torch.cuda.synchronize()
-    print(json.dumps({"kernel_only": name, "fmt": fmt_name, "N": N, "K": K, "launches": repeats,
-                      "y_finite": bool(torch.isfinite(y.float()).all())}))
+    print(json.dumps({"kernel_only": name, "fmt": fmt_name, "launches": repeats,
+                      "shapes": [[d.N, d.K] for d, *_ in mats],
+                      "y_finite": all(bool(torch.isfinite(m[4].float()).all()) for m in mats)}))
 
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kernel-only", choices=[n for n, _, _ in SHAPES], default=None,
-                    help="profiling case: one matrix of this shape, a few GEMV launches")
+    ap.add_argument("--kernel-only", choices=[n for n, _, _ in SHAPES] + ["layer"], default=None,
+                    help="profiling case: one matrix of this shape (or one decode layer), a few launches")
     ap.add_argument("--fmt", default="int4", help="format for --kernel-only")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)

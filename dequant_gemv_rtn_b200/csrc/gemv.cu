@@ -1,5 +1,5 @@
-// gemv.cu -- fused-dequant GEMV: the batch-1 tensor-core kernel for 4-bit
-// formats (mma.sync, below) and the CUDA-core multi-vector kernel (all formats).
+// gemv.cu -- fused-dequant GEMV on CUDA cores: the multi-vector kernel (all
+// formats; the batch-1 tensor-core kernel for 4-bit formats is in gemv1.cu).
 //
 // The decode-time kernel the RTN page ("Is (Selective) Round-To-Nearest
 // Quantization All You Need?", English abstract: token-generation throughput of
@@ -29,6 +29,7 @@
 //      INT8: PRMT into 0x64xx fp16 patterns and one subtract; FP16: direct.
 #include <mutex>
 #include "common.cuh"
+#include "gemv_common.cuh"
 #include "kernels.h"
 
 namespace qnt {
@@ -84,95 +85,6 @@ __device__ bool stage_activations(uint64_t* xbar, float* red, __half* xs, int K,
     __syncthreads();
   }
   return true;
-}
-
-// ------------------------------------------------------------------ metadata
-struct GroupMeta {
-  float s;   // INT4: s * 2^24; FP4 / RaZeR: s; AFPQ: s+
-  float t;   // INT4: s * z;   AFPQ: s-;  RaZeR: special value
-};
-
-// Metadata of group f (= row * groups_per_row + group) from global memory.
-template <int FMT>
-__device__ __forceinline__ GroupMeta group_meta(const uint8_t* meta, long z0, long f) {
-  GroupMeta g;
-  if (FMT == QNT_FP4_AFPQ) {
-    const uint32_t w = ldg_u32(meta + 4 * f);
-    g.s = h2f(w & 0xFFFFu);
-    g.t = h2f(w >> 16);
-    return g;
-  }
-  const float s = h2f(ldg_u16(meta + 2 * f));
-  if (FMT == QNT_INT4_ASYM) {
-    const uint32_t z = (ldg_u8(meta + z0 + f / 2) >> (4 * (f & 1))) & 15u;
-    g.s = s * 16777216.0f;     // 2^24 undoes the subnormal encoding
-    g.t = s * (float)z;
-  } else if (FMT == QNT_FP4_RAZER) {
-    const uint32_t sel = (ldg_u8(meta + z0 + f / 4) >> (2 * (f & 3))) & 3u;
-    const float sv = (sel & 2u) ? 8.0f : 5.0f;
-    g.s = s;
-    g.t = (sel & 1u) ? -sv : sv;
-  } else {
-    g.s = s;
-    g.t = 0.0f;
-  }
-  return g;
-}
-
-// The metadata of a CTA's rows, staged in shared memory: 16-byte-aligned
-// supersets of the scale plane (A bytes per group) and of the zero / selector
-// plane (B bits per group) that the rows [r_lo, r_hi) use.
-template <int FMT> struct MetaPlanes {
-  static constexpr int A = (FMT == QNT_FP4_AFPQ) ? 4 : 2;
-  static constexpr int B = (FMT == QNT_INT4_ASYM) ? 4 : (FMT == QNT_FP4_RAZER ? 2 : 0);
-};
-struct MetaWin { long a0, a1, b0, b1, bpl; };
-template <int FMT>
-__host__ __device__ inline MetaWin meta_window(long r_lo, long r_hi, long GK, long z0, long rows_cap) {
-  using MP = MetaPlanes<FMT>;
-  MetaWin m;
-  m.a0 = (MP::A * r_lo * GK) & ~15L;
-  m.a1 = (MP::A * r_hi * GK + 15) & ~15L;
-  m.bpl = (MP::A * rows_cap * GK + 32 + 15) & ~15L;   // plane B's offset in the staged copy
-  if (MP::B) {
-    m.b0 = (z0 + (r_lo * GK * MP::B) / 8) & ~15L;
-    m.b1 = (z0 + (r_hi * GK * MP::B + 7) / 8 + 15) & ~15L;
-  } else {
-    m.b0 = m.b1 = 0;
-  }
-  return m;
-}
-template <int FMT>
-__host__ __device__ inline size_t meta_stage_bytes(long rows_cap, long GK) {
-  using MP = MetaPlanes<FMT>;
-  const size_t a = ((size_t)MP::A * rows_cap * GK + 32 + 15) & ~size_t(15);
-  return a + (MP::B ? ((((size_t)rows_cap * GK * MP::B + 7) / 8 + 48 + 15) & ~size_t(15)) : 0);
-}
-// Metadata of group f from the staged copy.
-template <int FMT>
-__device__ __forceinline__ GroupMeta group_meta_s(const uint8_t* ms, const MetaWin& w, long z0, long f) {
-  GroupMeta g;
-  if (FMT == QNT_FP4_AFPQ) {
-    const uint32_t v = lds_u32(ms + (4 * f - w.a0));
-    g.s = h2f(v & 0xFFFFu);
-    g.t = h2f(v >> 16);
-    return g;
-  }
-  const float s = h2f(lds_u16(ms + (2 * f - w.a0)));
-  if (FMT == QNT_INT4_ASYM) {
-    const uint32_t z = (lds_u8(ms + w.bpl + (z0 + f / 2 - w.b0)) >> (4 * (f & 1))) & 15u;
-    g.s = s * 16777216.0f;
-    g.t = s * (float)z;
-  } else if (FMT == QNT_FP4_RAZER) {
-    const uint32_t sel = (lds_u8(ms + w.bpl + (z0 + f / 4 - w.b0)) >> (2 * (f & 3))) & 3u;
-    const float sv = (sel & 2u) ? 8.0f : 5.0f;
-    g.s = s;
-    g.t = (sel & 1u) ? -sv : sv;
-  } else {
-    g.s = s;
-    g.t = 0.0f;
-  }
-  return g;
 }
 
 // ------------------------------------------------------------------ per-chunk dot products
@@ -238,7 +150,6 @@ __device__ __forceinline__ float chunk_value(const GroupMeta& md, const float (&
   return md.s * (a[0] + a[1]);
 }
 
-__host__ __device__ inline size_t align16(size_t v) { return (v + 15) & ~size_t(15); }
 
 // Work ranges: 4-bit formats stream row groups of eight in ranges of 1024
 // weights (4 KB, one contiguous run of the layout); INT8 / FP16 stream pairs of
@@ -263,19 +174,6 @@ __host__ __device__ inline SmemSimt smem_simt_layout(int fmt, int MB, int K, int
   L.ms = align16(L.part + (size_t)MB * rows_cap * KR * 4);
   L.total = align16(L.ms + meta_bytes);
   return L;
-}
-
-// Rows of CTA b out of `grid`: 4-bit formats split whole row groups of eight.
-__host__ __device__ inline void simt_rows(int fmt, long N, int b, int grid, long* r_lo, long* r_hi) {
-  if (fmt == QNT_INT8_PERCHAN || fmt == QNT_FP16) {
-    *r_lo = (long)b * N / grid;
-    *r_hi = (long)(b + 1) * N / grid;
-  } else {
-    const long NG = (N + 7) / 8;
-    *r_lo = 8 * ((long)b * NG / grid);
-    const long hi = 8 * ((long)(b + 1) * NG / grid);
-    *r_hi = hi < N ? hi : N;
-  }
 }
 
 // ------------------------------------------------------------------ kernel
@@ -518,341 +416,6 @@ gemv_simt_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ 
   }
 }
 
-// ------------------------------------------------------------------ batch 1 on the tensor cores (mma.sync)
-// One activation vector, 4-bit formats.  A producer warp streams 8 KB runs of
-// the packed layout (one row group x 16 blocks of K, contiguous) into a
-// CTA-wide ring of slots with bulk copies; consumer warps take the runs in turn
-// and hand the multiply-adds to mma.sync m16n8k16 (fp16 inputs, fp32
-// accumulation) straight from the packed codes, so a lane spends five bit
-// operations and one MMA on eight weights.  Per-row partial sums of the runs are
-// combined in a fixed order (deterministic results).  Two CTAs per SM.
-//
-// Wait until ring slot `slot` holds item t and its bytes have landed, for
-// consumers that share one slot ring and each take every n-th item.  The tag
-// is read first: the producer writes t there only after the slot's previous
-// item has been consumed, so from then on the slot barrier's pending (or last
-// completed) phase is the one for t, and the parity wait cannot be met by a
-// phase two behind.  Bounded like every wait; false on timeout or abort.
-__device__ __forceinline__ bool ring_wait_item(volatile int* tag, uint64_t* full, int slot, int t, int nslot,
-                                               volatile int* abort_p) {
-  for (int it = 0; it < kMaxTries; ++it) {
-    if (tag[slot] == t) {
-      __threadfence_block();
-      return mbar_wait(full + slot, (uint32_t)(t / nslot) & 1u);
-    }
-    if (*abort_p) return false;
-    __nanosleep(256);
-  }
-  return false;
-}
-
-// One MMA covers the eight rows of a row group over 32 weights of each row.  Lane
-// t = 4g + r holds the 16-byte chunk r of row g of a block; word j of that chunk
-// feeds MMA j of the block.  A row g of the MMA's A operand is the row's first
-// half of the word's weights, row g + 8 its second half (two K segments of one
-// weight row); B column 2h + s holds the activations of segment s restricted to
-// group h of the block, so D[g][2h] + D[g + 8][2h + 1] is row g's dot product
-// over group h, found in lane 4g + h.  Which weights a word's halves hold is
-// fixed by the layout (INT4: nibbles at bits 0..3 and 4..7 of each fp16 half,
-// the latter 16x larger; FP4 family: e2m1 pairs), and the activation image
-// (xf, built once per CTA) puts each x where its weight's product lands.
-// Activations are scaled per block by an exact power of two that puts the block
-// maximum in [2^14, 2^15); B entries of INT4 nibbles at bits 4..7 carry x / 16.
-constexpr int kMmaConsumers = 7;
-constexpr int kMmaThreads = 32 * (1 + kMmaConsumers);
-constexpr int kMmaRangeBlocks = 16;                       // blocks per work item
-constexpr int kMmaItemBytes = kMmaRangeBlocks * 512;      // 8 KB: one row group x 16 blocks
-constexpr int kMmaMaxSlots = 12;
-constexpr int kMmaPrefetch = 1;                           // items requested before the activations
-constexpr int kMmaCtrl = 1024;                            // barriers, tags, 32 zero bytes at 768
-constexpr int kMmaSmemCap = 113 * 1024;                   // two CTAs per SM
-
-struct SmemMma { size_t ring, xraw, xf, xs2, part, ms, total; };
-__host__ __device__ inline SmemMma smem_mma_layout(int K, int G, int rows_cap, int nslot, size_t meta_bytes) {
-  const int KB = K / 128, KBR = (KB + kMmaRangeBlocks - 1) / kMmaRangeBlocks, GPB = 128 / G;
-  SmemMma L;
-  L.ring = kMmaCtrl;
-  L.xraw = L.ring + (size_t)nslot * kMmaItemBytes;
-  L.xf = align16(L.xraw + (size_t)K * 2);
-  L.xs2 = align16(L.xf + (size_t)K * 2);
-  L.part = align16(L.xs2 + (size_t)KB * GPB * 8);
-  L.ms = align16(L.part + (size_t)rows_cap * KBR * 4);
-  L.total = align16(L.ms + meta_bytes);
-  return L;
-}
-
-__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                          uint32_t b0, uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// Byte offset in the activation image of the B entry for block b, chunk r,
-// segment s, MMA j, half hf (b0: hf = 0, b1: hf = 1).  A lane reads its
-// (s, r) entry of a block with two 16-byte loads (MMAs 0, 1 and 2, 3).
-__device__ __forceinline__ uint32_t xf_off(int b, int r, int s, int j, int hf) {
-  return (uint32_t)(256 * b + 128 * (j >> 1) + 16 * (4 * s + r) + 8 * (j & 1) + 4 * hf);
-}
-
-// Activation image of blocks b0 and b1, built by one warp: lane l takes
-// x[128b + 4l .. 4l + 3] of each.  Within a chunk, the weight at offset o = 16 hf + 4j + 2s + e (INT4)
-// or 8j + 4hf + 2s + e (FP4 family) meets B half hf, segment s of MMA j.  Also
-// writes (c / 2^e, sum of x over group h) per (block, group) to xs2, c = 2^24
-// for INT4 (undoes the subnormal encoding), else 1.
-template <int FMT, int G>
-__device__ __forceinline__ void mma_build_x(uint32_t xraw, uint32_t xf, uint32_t xs2, int b0, int b1, int xbf16,
-                                            int lane) {
-  // two blocks per call (b1 < 0: none), so their shuffle reductions overlap
-  constexpr int GPB = 128 / G;
-  const int bb[2] = {b0, b1 >= 0 ? b1 : b0};
-  float v[2][4], am[2], sg[2];
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    const uint2 raw = lds64a(xraw + 256 * bb[q] + 8 * lane);
-    if (xbf16) {
-      v[q][0] = __uint_as_float(raw.x << 16); v[q][1] = __uint_as_float(raw.x & 0xFFFF0000u);
-      v[q][2] = __uint_as_float(raw.y << 16); v[q][3] = __uint_as_float(raw.y & 0xFFFF0000u);
-    } else {
-      v[q][0] = h2f(raw.x & 0xFFFFu); v[q][1] = h2f(raw.x >> 16);
-      v[q][2] = h2f(raw.y & 0xFFFFu); v[q][3] = h2f(raw.y >> 16);
-    }
-    am[q] = fmaxf(fmaxf(fabsf(v[q][0]), fabsf(v[q][1])), fmaxf(fabsf(v[q][2]), fabsf(v[q][3])));
-    sg[q] = (v[q][0] + v[q][1]) + (v[q][2] + v[q][3]);
-  }
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      am[q] = fmaxf(am[q], __shfl_xor_sync(0xffffffffu, am[q], o));
-      if (FMT == QNT_INT4_ASYM && o < G / 4) sg[q] += __shfl_xor_sync(0xffffffffu, sg[q], o);
-    }
-  }
-  const int r = lane >> 3, o = 4 * (lane & 7);
-  int j, hf;
-  if (FMT == QNT_INT4_ASYM) {
-    hf = o >> 4;
-    j = (o & 15) >> 2;
-  } else {
-    j = o >> 3;
-    hf = (o >> 2) & 1;
-  }
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    if (q == 1 && b1 < 0) break;
-    int e = 0;
-    if (am[q] > 0.0f && isfinite(am[q])) e = min(max(14 - (int)((__float_as_uint(am[q]) >> 23) & 255u) + 127, -126), 126);
-    const float f = __uint_as_float((uint32_t)(127 + e) << 23);
-    const float fs = (FMT == QNT_INT4_ASYM && hf) ? f * 0.0625f : f;   // INT4 bits 4..7 decode 16x too large
-    const __half2 p0 = __floats2half2_rn(v[q][0] * fs, v[q][1] * fs), p1 = __floats2half2_rn(v[q][2] * fs, v[q][3] * fs);
-    sts32a(xf + xf_off(bb[q], r, 0, j, hf), *reinterpret_cast<const uint32_t*>(&p0));
-    sts32a(xf + xf_off(bb[q], r, 1, j, hf), *reinterpret_cast<const uint32_t*>(&p1));
-    if ((lane & (G / 4 - 1)) == 0)
-      sts64fa(xs2 + 8 * (bb[q] * GPB + lane / (G / 4)),
-              __uint_as_float((uint32_t)(127 - e) << 23) * (FMT == QNT_INT4_ASYM ? 16777216.0f : 1.0f),
-              FMT == QNT_INT4_ASYM ? sg[q] : 0.0f);
-  }
-}
-
-template <int FMT, int G>
-__global__ void __launch_bounds__(kMmaThreads, 2)
-gemv4_mma_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ meta, long z0,
-                 const void* __restrict__ X, void* __restrict__ Y, int N, int K, int xbf16, int rows_cap,
-                 int nslot, int meta_bytes, int* d_status) {
-  constexpr int GPB = 128 / G;
-  constexpr int RB = kMmaRangeBlocks;
-  extern __shared__ __align__(1024) uint8_t smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
-  uint64_t* empty = full + kMmaMaxSlots;
-  uint64_t* xbar = empty + kMmaMaxSlots;
-  volatile int* abort_p = reinterpret_cast<volatile int*>(smem + 512);
-  volatile int* tag = reinterpret_cast<volatile int*>(smem + 640);   // item last issued into each slot
-  const SmemMma L = smem_mma_layout(K, G, rows_cap, nslot, (size_t)meta_bytes);
-  const uint32_t sbase = smem_addr(smem);
-  const uint32_t zero_a = sbase + 768, ring_a = sbase + (uint32_t)L.ring, xraw_a = sbase + (uint32_t)L.xraw;
-  const uint32_t xf_a = sbase + (uint32_t)L.xf, xs2_a = sbase + (uint32_t)L.xs2;
-  uint8_t* ring = smem + L.ring;
-  float* part = reinterpret_cast<float*>(smem + L.part);    // [rows_cap][KBR]
-  uint8_t* ms = smem + L.ms;
-  const int KB = K / 128, KBR = (KB + RB - 1) / RB, GK = K / G;
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  long r_lo, r_hi;
-  simt_rows(QNT_INT4_ASYM, N, blockIdx.x, gridDim.x, &r_lo, &r_hi);
-  const int nrows = (int)(r_hi - r_lo);
-  const int nitems = (nrows + 7) / 8 * KBR;
-  const MetaWin mw = meta_window<FMT>(r_lo, r_hi, GK, z0, rows_cap);
-
-  if (tid == 0) {
-    for (int i = 0; i < nslot; ++i) { mbar_init(full + i, 1); mbar_init(empty + i, 1); tag[i] = -1; }
-    mbar_init(xbar, 1);
-    *abort_p = 0;
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  }
-  if (tid < 8) reinterpret_cast<uint32_t*>(smem + 768)[tid] = 0u;   // the zero B entry
-  __syncthreads();
-
-  if (warp == 0) {
-    // ---------------------------------------------------------------- producer
-    if (lane == 0) {
-      const uint64_t pol = l2_evict_first_policy();
-      auto issue = [&](int t) {
-        const int u = t / KBR, br = t - u * KBR, slot = t % nslot;
-        const int nb = min(RB, KB - RB * br);
-        tag[slot] = t;   // before the arrive below, which releases it to the waiters
-        mbar_expect_tx(full + slot, (uint32_t)nb * 512u);
-        bulk_g2s_hint(ring + (size_t)slot * kMmaItemBytes, codes + (r_lo / 8 + u) * 4L * K + (long)br * RB * 512,
-                      (uint32_t)nb * 512u, full + slot, pol);
-      };
-      const bool stage_meta = meta_bytes > 0 && nrows > 0;
-      mbar_expect_tx(xbar, (uint32_t)K * 2u + (stage_meta ? (uint32_t)((mw.a1 - mw.a0) + (mw.b1 - mw.b0)) : 0u));
-      if (stage_meta) {
-        bulk_g2s(ms, meta + mw.a0, (uint32_t)(mw.a1 - mw.a0), xbar);
-        if (mw.b1 > mw.b0) bulk_g2s(ms + mw.bpl, meta + mw.b0, (uint32_t)(mw.b1 - mw.b0), xbar);
-      }
-      // a few weight runs before waiting for the previous kernel (weights do not
-      // depend on it); the activations are then queued ahead of the rest
-      int t = 0;
-      for (; t < nitems && t < nslot && t < kMmaPrefetch; ++t) issue(t);
-      asm volatile("griddepcontrol.wait;" ::: "memory");
-      bulk_g2s(smem + L.xraw, X, (uint32_t)K * 2u, xbar);
-      for (; t < nitems && t < nslot; ++t) issue(t);
-      for (; t < nitems; ++t) {
-        if (!mbar_wait(empty + t % nslot, (uint32_t)(t / nslot - 1) & 1u)) {
-          *abort_p = 1;
-          report(d_status, QNT_ERR_TIMEOUT);
-          break;
-        }
-        issue(t);
-      }
-      // drain: every issued copy has landed before the CTA exits
-      mbar_wait(xbar, 0);
-      for (int i = (t > nslot ? t - nslot : 0); i < t; ++i) mbar_wait(full + i % nslot, (uint32_t)(i / nslot) & 1u);
-    }
-  } else {
-    // ---------------------------------------------------------------- consumers
-    const int cw = warp - 1;
-    if (!mbar_wait(xbar, 0)) { *abort_p = 1; report(d_status, QNT_ERR_TIMEOUT); }
-    if (!*abort_p) {
-      for (int b = cw; b < KB; b += 2 * kMmaConsumers)
-        mma_build_x<FMT, G>(xraw_a, xf_a, xs2_a, b, b + kMmaConsumers < KB ? b + kMmaConsumers : -1, xbf16, lane);
-    }
-    asm volatile("bar.sync 1, %0;" :: "n"(32 * kMmaConsumers) : "memory");
-
-    const int g = lane >> 2, r = lane & 3;                       // A: row g, chunk r
-    const int hB = lane >> 3, sB = (lane >> 2) & 1;              // B: column 2 hB + sB
-    const bool bload = hB < GPB && r / (4 / GPB) == hB;
-    const uint32_t xb_a = bload ? xf_a + 16u * (uint32_t)(4 * sB + r) : zero_a;
-    const uint32_t xstride = bload ? 256u : 0u, xhi = bload ? 128u : 16u;   // lanes without B read zeros
-    const uint32_t coff = 64u * g + 16u * (uint32_t)(r ^ ((g >> 1) & 3));
-    const int re = r < GPB ? r : GPB - 1;                        // epilogue group (lanes r < GPB)
-    const int ra = r / (4 / GPB);                                // group of this lane's chunk
-    // staged metadata: plane A (scales) and plane B (zeros / selectors) by group index
-    const uint32_t msa = smem_addr(ms) - (uint32_t)mw.a0;
-    const uint32_t msb = smem_addr(ms) + (uint32_t)(mw.bpl + z0 - mw.b0);
-    for (int t = cw; t < nitems && !*abort_p; t += kMmaConsumers) {
-      const int u = t / KBR, br = t - u * KBR, slot = t % nslot;
-      const long row = r_lo + 8 * u + g;
-      const bool rowok = row < r_hi;
-      const bool ok = rowok && r < GPB;
-      const long rowm = rowok ? row : r_lo;                      // a row whose metadata is staged
-      const int nb = min(RB, KB - RB * br);
-      const int b0 = RB * br;
-      const int f0 = (int)(rowm * GK) + b0 * GPB;                // group of block b0 in this lane's row
-      if (!ring_wait_item(tag, full, slot, t, nslot, abort_p)) { *abort_p = 1; report(d_status, QNT_ERR_TIMEOUT); break; }
-      const uint32_t ca = ring_a + (uint32_t)slot * kMmaItemBytes + coff;
-      float yacc = 0.0f;
-#pragma unroll 2
-      for (int bi = 0; bi < nb; ++bi) {
-        const int b = b0 + bi;
-        const uint4 cv = lds128a(ca + 512u * bi);
-        const uint4 x0 = lds128a(xb_a + xstride * b), x1 = lds128a(xb_a + xstride * b + xhi);
-        const float2 sc = lds64fa(xs2_a + 8u * (uint32_t)(b * GPB + re));   // (c / 2^e, group sum of x)
-        const int fe = f0 + bi * GPB + re, fa = f0 + bi * GPB + ra;
-        float ms_s, ms_t = 0.0f;                                   // this lane's epilogue metadata
-        uint32_t sv16 = 0;
-        if (meta_bytes > 0) {
-          if (FMT == QNT_FP4_AFPQ) {
-            const uint32_t v = lds32a(msa + 4u * fe);
-            ms_s = h2f(v & 0xFFFFu);
-            ms_t = h2f(v >> 16);
-          } else {
-            ms_s = h2f(lds16a(msa + 2u * fe));
-          }
-          if (FMT == QNT_INT4_ASYM) ms_t = (float)((lds8a(msb + (uint32_t)(fe >> 1)) >> (4 * (fe & 1))) & 15u);
-          if (FMT == QNT_FP4_RAZER) {
-            const uint32_t sel = (lds8a(msb + (uint32_t)(fa >> 2)) >> (2 * (fa & 3))) & 3u;
-            sv16 = ((sel & 2u) ? 0x4800u : 0x4500u) | ((sel & 1u) ? 0x8000u : 0u);   // +-8 or +-5
-          }
-        } else {
-          const GroupMeta md = group_meta<FMT>(meta, z0, fe);
-          ms_s = md.s;
-          ms_t = md.t;
-          if (FMT == QNT_INT4_ASYM) { ms_s *= 1.0f / 16777216.0f; ms_t = ms_s == 0.0f ? 0.0f : md.t / ms_s; }
-          if (FMT == QNT_FP4_RAZER) sv16 = __half_as_ushort(__float2half_rn(group_meta<FMT>(meta, z0, fa).t));
-        }
-        const uint32_t w[4] = {cv.x, cv.y, cv.z, cv.w};
-        const uint32_t bx[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-        // two accumulator chains (MMAs 0, 2 and 1, 3)
-        float d[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
-        float dn[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          if (FMT == QNT_INT4_ASYM) {
-            const uint32_t w8 = w[j] >> 8;
-            mma_16816(d[j & 1], w[j] & 0x000F000Fu, w8 & 0x000F000Fu, w[j] & 0x00F000F0u, w8 & 0x00F000F0u,
-                      bx[2 * j], bx[2 * j + 1]);
-          } else {
-            uint32_t h[4];
-            cvt_e2m1x8(w[j], h[0], h[1], h[2], h[3]);
-            if (FMT == QNT_FP4_RAZER) {
-              // codes 0b1000 (decoded as -0) take the group's special value
-              const uint32_t tt = (w[j] & 0x77777777u) + 0x77777777u;
-              const uint32_t spec = lop3<0x20>(w[j], tt, 0x88888888u);
-#pragma unroll
-              for (int pp = 0; pp < 4; ++pp) {
-                if (spec & (0x8u << (8 * pp))) h[pp] = (h[pp] & 0xFFFF0000u) | sv16;
-                if (spec & (0x80u << (8 * pp))) h[pp] = (h[pp] & 0x0000FFFFu) | (sv16 << 16);
-              }
-            }
-            if (FMT == QNT_FP4_AFPQ) {
-              uint32_t hp[4], hn[4];
-#pragma unroll
-              for (int pp = 0; pp < 4; ++pp) { hp[pp] = hmax2(h[pp], 0u); hn[pp] = hsub2(h[pp], hp[pp]); }
-              mma_16816(d[j & 1], hp[0], hp[1], hp[2], hp[3], bx[2 * j], bx[2 * j + 1]);
-              mma_16816(dn[j & 1], hn[0], hn[1], hn[2], hn[3], bx[2 * j], bx[2 * j + 1]);
-            } else {
-              mma_16816(d[j & 1], h[0], h[1], h[2], h[3], bx[2 * j], bx[2 * j + 1]);
-            }
-          }
-        }
-        const float v = (d[0][0] + d[0][3]) + (d[1][0] + d[1][3]);
-        float c;
-        if (FMT == QNT_INT4_ASYM) {
-          c = ms_s * (sc.x * v - ms_t * sc.y);
-        } else if (FMT == QNT_FP4_AFPQ) {
-          c = sc.x * (ms_s * v + ms_t * ((dn[0][0] + dn[0][3]) + (dn[1][0] + dn[1][3])));
-        } else {
-          c = ms_s * sc.x * v;
-        }
-        yacc += ok ? c : 0.0f;
-      }
-      __syncwarp();
-      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_addr(empty + slot)) : "memory");
-      if (GPB > 1) yacc += __shfl_xor_sync(0xffffffffu, yacc, 1);
-      if (GPB > 2) yacc += __shfl_xor_sync(0xffffffffu, yacc, 2);
-      if (r == 0 && rowok) part[(size_t)(8 * u + g) * KBR + br] = yacc;
-    }
-  }
-  __syncthreads();
-  for (int rl = tid; rl < nrows; rl += kMmaThreads) {
-    float v = 0.0f;
-    for (int br = 0; br < KBR; ++br) v += part[(size_t)rl * KBR + br];
-    if (xbf16) reinterpret_cast<__nv_bfloat16*>(Y)[r_lo + rl] = __float2bfloat16_rn(v);
-    else reinterpret_cast<__half*>(Y)[r_lo + rl] = __float2half_rn(v);
-  }
-}
-
 // ------------------------------------------------------------------ launchers
 int num_sms() {
   static int sms[64] = {0};
@@ -975,67 +538,6 @@ int gemv_max_mb(const qnt_desc& d) {
   return best;
 }
 
-template <int FMT, int G>
-static cudaError_t launch_mma(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
-                              int xbf16, int* st, cudaStream_t s, bool* handled) {
-  // two CTAs per SM where the shared memory allows it: the row groups are split
-  // over twice the SM count
-  const int NG = (d.N + 7) / 8;
-  const int grid = NG < 2 * num_sms() ? NG : 2 * num_sms();
-  const int rows_cap = 8 * ((NG + grid - 1) / grid);
-  auto total = [&](int ns, size_t mb) { return smem_mma_layout(d.K, G, rows_cap, ns, mb).total; };
-  size_t mb = meta_stage_bytes<FMT>(rows_cap, d.K / G);
-  int nslot = 0;
-  for (size_t cap : {(size_t)kMmaSmemCap, (size_t)kMaxDynSmem}) {
-    for (size_t m : {mb, (size_t)0}) {
-      for (int ns = kMmaMaxSlots; ns >= 2 && nslot == 0; --ns)
-        if (total(ns, m) <= cap) { nslot = ns; mb = m; }
-      if (nslot) break;
-    }
-    if (nslot) break;
-  }
-  if (nslot == 0) return cudaSuccess;   // not handled
-  const size_t smem = total(nslot, mb);
-  auto kfn = gemv4_mma_kernel<FMT, G>;
-  cudaError_t e = configure_smem(reinterpret_cast<const void*>(kfn));
-  if (e != cudaSuccess) return e;
-  *handled = true;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kMmaThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kfn, static_cast<const uint8_t*>(codes), static_cast<const uint8_t*>(meta), z0, X, Y,
-                            d.N, d.K, xbf16, rows_cap, nslot, (int)mb, st);
-}
-
-// One activation vector, 4-bit formats: the tensor-core kernel above.
-// *handled = false when it does not take the shape.
-cudaError_t launch_gemv4_one(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
-                             int xbf16, int* st, cudaStream_t s, bool* handled) {
-  *handled = false;
-#define QNT_RG(FMT)                                                                          \
-  switch (d.group) {                                                                         \
-    case 32: return launch_mma<FMT, 32>(d, codes, meta, z0, X, Y, xbf16, st, s, handled);    \
-    case 64: return launch_mma<FMT, 64>(d, codes, meta, z0, X, Y, xbf16, st, s, handled);    \
-    default: return launch_mma<FMT, 128>(d, codes, meta, z0, X, Y, xbf16, st, s, handled);   \
-  }
-  switch (d.fmt) {
-    case QNT_INT4_ASYM: QNT_RG(QNT_INT4_ASYM)
-    case QNT_FP4_E2M1: QNT_RG(QNT_FP4_E2M1)
-    case QNT_FP4_AFPQ: QNT_RG(QNT_FP4_AFPQ)
-    case QNT_FP4_RAZER: QNT_RG(QNT_FP4_RAZER)
-    default: return cudaSuccess;
-  }
-#undef QNT_RG
-}
-
-// Y[m] = W x[m] for m < M on CUDA cores, in passes of up to 8 vectors.
 cudaError_t launch_gemv_simt(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
                              int M, int xbf16, int* st, cudaStream_t s) {
   const int mbmax = gemv_max_mb(d);

@@ -23,11 +23,20 @@ cudaError_t launch_gemv_simt(const qnt_desc& d, const void* codes, const void* m
                              void* Y, int M, int xbf16, int* st, cudaStream_t s);
 
 // y = W x for one activation vector, 4-bit formats, on the tensor cores with
-// mma.sync straight from the packed codes (gemv.cu).  *handled = false when it
+// mma.sync straight from the packed codes (gemv1.cu).  *handled = false when it
 // does not apply (the activation vector and a weight ring do not fit in shared
 // memory).
 cudaError_t launch_gemv4_one(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
                              int xbf16, int* st, cudaStream_t s, bool* handled);
+
+// A sequence of batch-1 GEMVs (4-bit formats) in one cooperative launch
+// (gemv1.cu); clears the workspace first.  *handled = false when the
+// activation vector and a weight ring do not fit in shared memory.
+cudaError_t launch_gemv_seq(const qnt_seq_step* steps, int n, int xbf16, void* work, int* st, cudaStream_t s,
+                            bool* handled);
+
+// An empty kernel: the next kernel in the stream cannot overlap the ones before it.
+cudaError_t launch_stream_fence(cudaStream_t s);
 
 // Y[m] = W x[m] for m < M on the tensor cores (gemv_tc.cu).  Returns with
 // *handled = false, launching nothing, when the tensor-core kernel does not

@@ -2,6 +2,7 @@
 // kernel dispatch.  Nothing here allocates memory; every launch goes to the
 // caller's stream.
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <cuda_runtime.h>
 #include "qnt.h"
@@ -10,6 +11,15 @@
 #include "kernels.h"
 
 namespace {
+
+thread_local char g_last_error[256] = "";
+
+// Map a CUDA status to the ABI's code, remembering the text of a failure.
+int cuda_rc(cudaError_t e) {
+  if (e == cudaSuccess) return QNT_OK;
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+  return QNT_ERR_CUDA;
+}
 
 bool is_4bit(int f) { return f == QNT_INT4_ASYM || f == QNT_FP4_E2M1 || f == QNT_FP4_AFPQ || f == QNT_FP4_RAZER; }
 
@@ -109,6 +119,8 @@ size_t qnt_meta_bytes(const qnt_desc* d) {
   }
 }
 
+const char* qnt_last_error(void) { return g_last_error; }
+
 const char* qnt_strerror(int code) {
   switch (code) {
     case QNT_OK: return "ok";
@@ -133,35 +145,67 @@ int qnt_quantize(const qnt_desc* desc, const float* d_W, void* d_codes, void* d_
   if (desc->fmt == QNT_INT4_ASYM || desc->fmt == QNT_FP4_RAZER) {
     // the zero / selector plane is filled with atomic ORs: clear it first
     const size_t tail = qnt_meta_bytes(desc) - (size_t)z0;   /* a multiple of 16 bytes */
-    if (cudaMemsetAsync(static_cast<uint8_t*>(d_meta) + z0, 0, tail, s) != cudaSuccess)
-      return QNT_ERR_CUDA;
+    const int rc = cuda_rc(cudaMemsetAsync(static_cast<uint8_t*>(d_meta) + z0, 0, tail, s));
+    if (rc != QNT_OK) return rc;
   }
-  return qnt::launch_quantize(*desc, d_W, d_codes, d_meta, z0, d_status, s) == cudaSuccess ? QNT_OK : QNT_ERR_CUDA;
+  const int rc = cuda_rc(qnt::launch_quantize(*desc, d_W, d_codes, d_meta, z0, d_status, s));
+  if (rc != QNT_OK) return rc;
+  // a GEMV right after this call requests the codes before it waits for the
+  // preceding kernel: put a kernel in between that starts only after this one
+  return cuda_rc(qnt::launch_stream_fence(s));
+}
+
+size_t qnt_gemv_seq_work_bytes(int nsteps) {
+  if (nsteps < 1 || nsteps > QNT_SEQ_MAX_STEPS) return 0;
+  return (size_t)round_up(4L * (nsteps + 1), 16);   // a counter per step, then an abort word
+}
+
+int qnt_gemv_seq(const qnt_seq_step* steps, int nsteps, int xdtype, void* d_work, int* d_status, void* stream) {
+  if (!steps || nsteps < 1 || nsteps > QNT_SEQ_MAX_STEPS) return QNT_ERR_ARG;
+  if (xdtype != QNT_F16 && xdtype != QNT_BF16) return QNT_ERR_ARG;
+  if (!d_work) return QNT_ERR_ARG;
+  for (int i = 0; i < nsteps; ++i) {
+    const qnt_seq_step& t = steps[i];
+    const int e = check(&t.desc);
+    if (e != QNT_OK) return e;
+    if (!is_4bit(t.desc.fmt) || t.desc.fmt != steps[0].desc.fmt || t.desc.group != steps[0].desc.group)
+      return QNT_ERR_ARG;
+    if (t.wait < 0 || t.wait > i) return QNT_ERR_ARG;
+    if (t.desc.K > QNT_MAX_GEMV_K) return QNT_ERR_SHAPE;
+    if (!t.codes || !t.meta || !t.x || !t.y) return QNT_ERR_ARG;
+    if (!aligned16(t.codes) || !aligned16(t.meta) || !aligned16(t.x) || !aligned16(t.y)) return QNT_ERR_ALIGN;
+  }
+  if (!aligned16(d_work)) return QNT_ERR_ALIGN;
+  bool handled = false;
+  const int rc = cuda_rc(qnt::launch_gemv_seq(steps, nsteps, xdtype == QNT_BF16, d_work, d_status,
+                                              static_cast<cudaStream_t>(stream), &handled));
+  if (rc != QNT_OK) return rc;
+  return handled ? QNT_OK : QNT_ERR_SHAPE;
 }
 
 int qnt_gemm(const qnt_desc* desc, const void* d_codes, const void* d_meta, const void* d_X, void* d_Y, int M,
              int xdtype, int* d_status, void* stream) {
   int e = check(desc);
   if (e != QNT_OK) return e;
+  if (desc->K > QNT_MAX_GEMV_K) return QNT_ERR_SHAPE;
   if (M < 1 || M > 128) return QNT_ERR_ARG;
   if (xdtype != QNT_F16 && xdtype != QNT_BF16) return QNT_ERR_ARG;
   if (!d_codes || !d_X || !d_Y || (desc->fmt != QNT_FP16 && !d_meta)) return QNT_ERR_ARG;
   if (!aligned16(d_codes) || !aligned16(d_X) || !aligned16(d_Y) || (d_meta && !aligned16(d_meta))) return QNT_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return dispatch_gemm(*desc, d_codes, d_meta, d_X, d_Y, M, xdtype == QNT_BF16, d_status, s) == cudaSuccess
-             ? QNT_OK : QNT_ERR_CUDA;
+  return cuda_rc(dispatch_gemm(*desc, d_codes, d_meta, d_X, d_Y, M, xdtype == QNT_BF16, d_status, s));
 }
 
 int qnt_gemv(const qnt_desc* desc, const void* d_codes, const void* d_meta, const void* d_x, void* d_y, int xdtype,
              int* d_status, void* stream) {
   int e = check(desc);
   if (e != QNT_OK) return e;
+  if (desc->K > QNT_MAX_GEMV_K) return QNT_ERR_SHAPE;
   if (xdtype != QNT_F16 && xdtype != QNT_BF16) return QNT_ERR_ARG;
   if (!d_codes || !d_x || !d_y || (desc->fmt != QNT_FP16 && !d_meta)) return QNT_ERR_ARG;
   if (!aligned16(d_codes) || !aligned16(d_x) || !aligned16(d_y) || (d_meta && !aligned16(d_meta))) return QNT_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return dispatch_gemm(*desc, d_codes, d_meta, d_x, d_y, 1, xdtype == QNT_BF16, d_status, s) == cudaSuccess
-             ? QNT_OK : QNT_ERR_CUDA;
+  return cuda_rc(dispatch_gemm(*desc, d_codes, d_meta, d_x, d_y, 1, xdtype == QNT_BF16, d_status, s));
 }
 
 }  // extern "C"

@@ -283,6 +283,15 @@ static cudaError_t launch_q4(const qnt_desc& d, const float* W, void* codes, voi
   return cudaGetLastError();
 }
 
+__global__ void stream_fence_kernel() {}
+
+// An empty kernel: a GEMV enqueued after it starts early only relative to this
+// kernel, which itself starts after everything before it has completed.
+cudaError_t launch_stream_fence(cudaStream_t s) {
+  stream_fence_kernel<<<1, 32, 0, s>>>();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quantize(const qnt_desc& d, const float* W, void* codes, void* meta, long z0, int* st, cudaStream_t s) {
   switch (d.fmt) {
     case QNT_INT4_ASYM: return launch_q4<QNT_INT4_ASYM>(d, W, codes, meta, z0, st, s);

@@ -22,8 +22,17 @@ FORMATS = {"int4": QNT_INT4_ASYM, "fp4": QNT_FP4_E2M1, "afpq": QNT_FP4_AFPQ, "ra
            "int8": QNT_INT8_PERCHAN, "fp16": QNT_FP16}
 
 
+QNT_MAX_GEMV_K = 65536
+QNT_SEQ_MAX_STEPS = 256
+
+
 class qnt_desc(ctypes.Structure):
     _fields_ = [("fmt", ctypes.c_int32), ("N", ctypes.c_int32), ("K", ctypes.c_int32), ("group", ctypes.c_int32)]
+
+
+class qnt_seq_step(ctypes.Structure):
+    _fields_ = [("desc", qnt_desc), ("codes", ctypes.c_void_p), ("meta", ctypes.c_void_p), ("x", ctypes.c_void_p),
+                ("y", ctypes.c_void_p), ("wait", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 def _load():
@@ -40,12 +49,15 @@ def _load():
         "qnt_quantize": (I, [D, P, P, P, P, P]),
         "qnt_gemv": (I, [D, P, P, P, P, I, P, P]),
         "qnt_gemm": (I, [D, P, P, P, P, I, I, P, P]),
+        "qnt_gemv_seq_work_bytes": (Z, [I]),
+        "qnt_gemv_seq": (I, [ctypes.POINTER(qnt_seq_step), I, I, P, P, P]),
         "qnt_table_create": (P, [I, I]),
         "qnt_table_set": (I, [P, ctypes.c_char_p, I, I]),
         "qnt_table_lookup": (I, [P, ctypes.c_char_p, ctypes.POINTER(I), ctypes.POINTER(I)]),
         "qnt_table_size": (I, [P]),
         "qnt_table_destroy": (None, [P]),
         "qnt_strerror": (ctypes.c_char_p, [I]),
+        "qnt_last_error": (ctypes.c_char_p, []),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -58,7 +70,8 @@ lib = _load()
 
 class QntError(RuntimeError):
     def __init__(self, code: int, what: str):
-        super().__init__(f"{what}: {qnt_strerror(code)} (code {code})")
+        extra = f" [{qnt_last_error()}]" if code == QNT_ERR_CUDA else ""
+        super().__init__(f"{what}: {qnt_strerror(code)} (code {code}){extra}")
         self.code = code
 
 
@@ -99,6 +112,10 @@ def qnt_strerror(code: int) -> str:
     return lib.qnt_strerror(int(code)).decode()
 
 
+def qnt_last_error() -> str:
+    return lib.qnt_last_error().decode()
+
+
 def qnt_check_desc(d: qnt_desc) -> int:
     return lib.qnt_check_desc(ctypes.byref(d))
 
@@ -127,6 +144,27 @@ def qnt_gemm(d: qnt_desc, codes, meta, X, Y, M: int, xdtype: int = QNT_F16, stat
     rc = lib.qnt_gemm(ctypes.byref(d), _ptr(codes), _ptr(meta), _ptr(X), _ptr(Y), int(M), int(xdtype), _ptr(status),
                       _stream(stream))
     return _check(rc, "qnt_gemm") if check else rc
+
+
+def seq_steps(items) -> ctypes.Array:
+    """Build a host array of qnt_seq_step from (desc, codes, meta, x, y, wait) tuples."""
+    arr = (qnt_seq_step * len(items))()
+    for i, (d, codes, meta, x, y, wait) in enumerate(items):
+        arr[i].desc = d
+        arr[i].codes, arr[i].meta, arr[i].x, arr[i].y = _ptr(codes), _ptr(meta), _ptr(x), _ptr(y)
+        arr[i].wait = int(wait)
+        arr[i].reserved = 0
+    return arr
+
+
+def qnt_gemv_seq_work_bytes(nsteps: int) -> int:
+    return lib.qnt_gemv_seq_work_bytes(int(nsteps))
+
+
+def qnt_gemv_seq(steps, xdtype: int, work, status=None, stream=None, check=True) -> int:
+    """steps: a ctypes array from seq_steps() (host memory)."""
+    rc = lib.qnt_gemv_seq(steps, len(steps), int(xdtype), _ptr(work), _ptr(status), _stream(stream))
+    return _check(rc, "qnt_gemv_seq") if check else rc
 
 
 class qnt_table:

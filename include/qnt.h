@@ -49,7 +49,11 @@
 extern "C" {
 #endif
 
-#define QNT_VERSION 1
+#define QNT_VERSION 2
+
+/* Largest K that qnt_gemv, qnt_gemm and qnt_gemv_seq accept (the activation
+ * vector is staged in shared memory); qnt_quantize accepts K up to 2^20. */
+#define QNT_MAX_GEMV_K 65536
 
 /* Weight formats.  h(.) = round-to-nearest-even to fp16; every quotient below
  * is one IEEE binary32 division; rint = round half to even; a scale that
@@ -91,7 +95,8 @@ typedef enum { QNT_F16 = 0, QNT_BF16 = 1 } qnt_dtype;
 enum {
   QNT_OK = 0,
   QNT_ERR_ARG = 1,       /* null pointer, unknown format / dtype, M out of range */
-  QNT_ERR_SHAPE = 2,     /* N < 1, K % 128 != 0, group not in {32,64,128} (4-bit) or != K */
+  QNT_ERR_SHAPE = 2,     /* N < 1, K % 128 != 0, group not in {32,64,128} (4-bit) or != K,
+                            K > QNT_MAX_GEMV_K for a GEMV / GEMM */
   QNT_ERR_ALIGN = 3,     /* a buffer is not 16-byte aligned */
   QNT_ERR_CUDA = 4,      /* the kernel launch failed */
   QNT_ERR_TIMEOUT = 5,   /* (device) a bounded wait for an asynchronous copy expired */
@@ -158,7 +163,9 @@ int qnt_check_desc(const qnt_desc* desc);
  *   d_codes    device, qnt_codes_bytes(desc) bytes, written.
  *   d_meta     device, qnt_meta_bytes(desc) bytes, written (may be NULL for FP16).
  *   d_status   device int or NULL: QNT_ERR_NONFINITE / QNT_ERR_RANGE.
- * Bit-exact with the definitions above.
+ * Bit-exact with the definitions above.  The call ends with an empty kernel on
+ * the stream, so that a GEMV enqueued right after it (which requests its codes
+ * and metadata before waiting for the preceding kernel, see qnt_gemv) sees them.
  */
 int qnt_quantize(const qnt_desc* desc, const float* d_W, void* d_codes, void* d_meta,
                  int* d_status, void* stream);
@@ -170,6 +177,13 @@ int qnt_quantize(const qnt_desc* desc, const float* d_W, void* d_codes, void* d_
  *   d_x        device, [K] fp16 or bf16 (xdtype).
  *   d_y        device, [N] in the same type, written.
  *   d_status   device int or NULL: QNT_ERR_TIMEOUT if a staging wait expires.
+ * Ordering (programmatic dependent launch): the GEMV kernels of qnt_gemv and
+ * qnt_gemm start while the preceding kernel on the stream is still running and
+ * request their codes and metadata at once; only the reads of x and the writes
+ * of y wait for that kernel to complete.  So the kernel IMMEDIATELY preceding
+ * the call on the stream must not write d_codes or d_meta.  qnt_quantize
+ * complies (it ends with an empty kernel); after any other kernel that writes
+ * the weights, enqueue another kernel or a copy in between, or synchronize.
  * Accuracy: |y - y_exact| <= 4e-3 * sum_k |dq(n,k) x[k]| per element.  Every
  * product is formed from exact fp16 operands and accumulated in fp32 (on the
  * CUDA cores exactly; on the tensor cores, which take batch 1 and larger
@@ -191,6 +205,55 @@ int qnt_gemm(const qnt_desc* desc, const void* d_codes, const void* d_meta,
              const void* d_X, void* d_Y, int M, int xdtype, int* d_status, void* stream);
 
 /*
+ * Sequences of batch-1 GEMVs in one launch: the linear layers of a decode step
+ * (token generation with fused-dequant kernels, RTN and RaZeR pages' English
+ * abstracts) run one after another on one activation vector each.  One
+ * persistent kernel streams the weights of every step back to back; a step
+ * with wait = k reads its x only after step i - k and every step before it
+ * have written their y, so x may be (part of) one of those y.  (A decode layer:
+ * o waits 1 for qkv, gate 1 for o, up 2 for o, down 1 for up.)
+ */
+#define QNT_SEQ_MAX_STEPS 256
+
+typedef struct {
+  qnt_desc desc;       /* 4-bit format, N, K, group: format and group equal in every step */
+  const void* codes;   /* device, this step's packed codes */
+  const void* meta;    /* device, its metadata */
+  const void* x;       /* device, [K] activations (fp16 or bf16, as xdtype) */
+  void* y;             /* device, [N] output, same type; written */
+  int32_t wait;        /* k >= 1: read x after step i - k and every step before it
+                          have written their y (x may be any of those y); 0: x is
+                          not written by any earlier step of this call.  0 <= k <= i. */
+  int32_t reserved;    /* 0 */
+} qnt_seq_step;
+
+/* Bytes of the workspace qnt_gemv_seq needs for nsteps steps (0 if nsteps is
+ * out of range). */
+size_t qnt_gemv_seq_work_bytes(int nsteps);
+
+/*
+ * qnt_gemv_seq -- y_i = W_i x_i for the steps i = 0 .. nsteps-1, in order.
+ *   steps      HOST array of nsteps step descriptors (1 <= nsteps <=
+ *              QNT_SEQ_MAX_STEPS); read during the call only.
+ *   d_work     device, qnt_gemv_seq_work_bytes(nsteps) bytes, 16-byte aligned,
+ *              owned by the caller: per-step completion counters.  The call
+ *              clears it on the stream before the kernel; two calls that may
+ *              run at the same time need two workspaces.
+ *   d_status   device int or NULL: QNT_ERR_TIMEOUT if a wait expires (a step's
+ *              dependency, a staging copy).
+ * Step 0 starts after the preceding work on the stream has completed.  The y of
+ * a step must not overlap any other step's y, x, codes or metadata except as
+ * the x of a later step marked `wait`.  Accuracy as qnt_gemv.  The kernel keeps
+ * one CTA on every SM for its whole duration (a cooperative launch);
+ * QNT_ERR_CUDA if the GPU cannot host it.  QNT_ERR_ARG: nsteps out of range,
+ * a null pointer, a format that is not 4-bit, formats / groups that differ
+ * between steps, or wait outside 0..i; QNT_ERR_SHAPE / QNT_ERR_ALIGN as for
+ * qnt_gemv, and QNT_ERR_SHAPE when a step's activations and staged metadata
+ * do not fit in shared memory.
+ */
+int qnt_gemv_seq(const qnt_seq_step* steps, int nsteps, int xdtype, void* d_work, int* d_status, void* stream);
+
+/*
  * Selective precision (RTN page: raise the precision format of chosen layers
  * and modules).  A host-side table of ordered rules; qnt_table_lookup returns
  * the format and group of the first rule whose pattern matches the module name
@@ -207,6 +270,11 @@ void qnt_table_destroy(qnt_table* t);
 
 /* Static description of an error code. */
 const char* qnt_strerror(int code);
+
+/* After a call returned QNT_ERR_CUDA: the CUDA runtime's name and description
+ * of the error, for the calling host thread ("" if none).  The text stays
+ * valid until the thread's next failing call. */
+const char* qnt_last_error(void);
 
 /* Library version (QNT_VERSION of the build). */
 int qnt_version(void);

@@ -40,7 +40,7 @@ def test_exports_every_declared_symbol(q):
 
 
 def test_version_and_strerror(q):
-    assert q.qnt_version() == 1
+    assert q.qnt_version() == 2
     for c in range(8):
         assert q.qnt_strerror(c)
     assert "unknown" in q.qnt_strerror(99)
@@ -121,3 +121,48 @@ def test_glob_edge_cases(q):
     assert t.lookup("aXXbYY")[0] == q.QNT_FP4_E2M1
     assert t.lookup("")[0] == q.QNT_FP16
     assert t.lookup("abcc")[0] == q.QNT_INT8_PERCHAN
+
+
+def test_gemv_k_bound(q):
+    """K above QNT_MAX_GEMV_K (the activation vector is staged in shared memory)
+    is a shape error for the GEMV calls, not a launch failure; quantize takes it."""
+    A = 1 << 20
+    big = q.desc(1, 64, q.QNT_MAX_GEMV_K + 128, 128)
+    assert q.qnt_check_desc(big) == q.QNT_OK
+    assert q.qnt_gemv(big, A, A, A, A, check=False, stream=0) == q.QNT_ERR_SHAPE
+    assert q.qnt_gemm(big, A, A, A, A, 4, check=False, stream=0) == q.QNT_ERR_SHAPE
+    steps = q.seq_steps([(big, A, A, A, A, 0)])
+    assert q.qnt_gemv_seq(steps, q.QNT_F16, A, check=False, stream=0) == q.QNT_ERR_SHAPE
+
+
+def test_seq_work_bytes(q):
+    assert q.qnt_gemv_seq_work_bytes(0) == 0
+    assert q.qnt_gemv_seq_work_bytes(q.QNT_SEQ_MAX_STEPS + 1) == 0
+    for n in (1, 3, 4, 160, q.QNT_SEQ_MAX_STEPS):
+        b = q.qnt_gemv_seq_work_bytes(n)
+        assert b >= 4 * (n + 1) and b % 16 == 0
+
+
+def test_seq_rejects_bad_arguments_without_launching(q):
+    A = 1 << 20
+    d4 = q.desc(1, 64, 256, 128)
+    ok = (d4, A, A, A, A, 0)
+    assert q.qnt_gemv_seq(q.seq_steps([]), 0, A, check=False, stream=0) == q.QNT_ERR_ARG
+    assert q.qnt_gemv_seq(q.seq_steps([ok] * (q.QNT_SEQ_MAX_STEPS + 1)), 0, A, check=False, stream=0) == q.QNT_ERR_ARG
+    cases = [
+        ([ok, (q.desc(2, 64, 256, 128), A, A, A, A, 1)], 0, A, q.QNT_ERR_ARG),     # formats differ
+        ([ok, (q.desc(1, 64, 256, 64), A, A, A, A, 1)], 0, A, q.QNT_ERR_ARG),      # groups differ
+        ([(d4, A, A, A, A, 0), ok, (d4, A, A, A, A, 2)], 0, None, q.QNT_ERR_ARG),  # (valid waits, no workspace)
+        ([(q.desc(5, 64, 256, 256), A, A, A, A, 0)], 0, A, q.QNT_ERR_ARG),         # not 4-bit
+        ([ok, (d4, A, A, None, A, 1)], 0, A, q.QNT_ERR_ARG),                       # null x
+        ([ok, (d4, A, A, A, A, 2)], 0, A, q.QNT_ERR_ARG),                          # waits past step 0
+        ([(d4, A, A, A, A, 1)], 0, A, q.QNT_ERR_ARG),                              # step 0 cannot wait
+        ([ok, (d4, A, A, A, A, -1)], 0, A, q.QNT_ERR_ARG),                         # negative wait
+        ([ok], 7, A, q.QNT_ERR_ARG),                                               # dtype
+        ([ok], 0, None, q.QNT_ERR_ARG),                                            # no workspace
+        ([ok, (d4, A, A + 8, A, A, 1)], 0, A, q.QNT_ERR_ALIGN),                    # metadata alignment
+        ([ok], 0, A + 4, q.QNT_ERR_ALIGN),                                         # workspace alignment
+        ([(q.desc(1, 64, 100, 32), A, A, A, A, 0)], 0, A, q.QNT_ERR_SHAPE),        # K % 128
+    ]
+    for items, xdt, work, want in cases:
+        assert q.qnt_gemv_seq(q.seq_steps(items), xdt, work, check=False, stream=0) == want, (items, want)

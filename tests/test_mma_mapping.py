@@ -210,3 +210,63 @@ def test_activation_image_offsets_agree_between_builder_and_reader():
                         assert off == read(b, r, s, 2 * j + hf)
                         offsets.add(off)
     assert sorted(offsets) == list(range(0, 3 * 256, 4))      # 256 bytes per block, no overlap
+
+
+# ------------------------------------------------------------------ several blocks per set of accumulators
+def emulate_set(fmt, qs, xs, G, q, NQ):
+    """The kernel's set scheme: a set of S = 4 / GPB blocks (q + NQ i, i < S),
+    one accumulator D_i per block, all fed the same B registers.  Lane t = 4g + r
+    takes B column pair hp = t / 8, i.e. block q + NQ (hp / GPB), group hp % GPB,
+    and loads its entry only if its chunk r lies in that group (G = 128: every
+    lane).  The epilogue of lane 4g + r reads D_{r / GPB}[g][2r] +
+    D_{r / GPB}[g+8][2r+1]: row g's dot product over block q + NQ (r / GPB),
+    group r % GPB.  qs / xs map a block index to its codes / activations."""
+    GPB = 128 // G
+    S = 4 // GPB
+    ents = {b: b_entries(fmt, xs[b], G) for b in xs}
+    acc = [np.zeros((16, 8)) for _ in range(S)]
+    for i in range(S):
+        words = pack_block(fmt, qs[q + NQ * i])
+        for j in range(4):
+            A = np.zeros((16, 8 * 2))
+            B = np.zeros((16, 8))
+            for t in range(32):
+                g, r = t // 4, t % 4
+                w = int(words[4 * (4 * g + (r ^ ((g // 2) % 4))) + j])
+                a = a_fragments(fmt, w)
+                A[g, 2 * r:2 * r + 2] = a[0]
+                A[g + 8, 2 * r:2 * r + 2] = a[1]
+                A[g, 2 * r + 8:2 * r + 10] = a[2]
+                A[g + 8, 2 * r + 8:2 * r + 10] = a[3]
+                n, hp, sB = t // 4, t // 8, (t // 4) % 2
+                if (r * GPB) // 4 == hp % GPB:
+                    bb = q + NQ * (hp // GPB)
+                    B[2 * r:2 * r + 2, n] = ents[bb][sB, r, j, 0]
+                    B[2 * r + 8:2 * r + 10, n] = ents[bb][sB, r, j, 1]
+            acc[i] += A @ B
+    return np.array([acc[(t % 4) // GPB][t // 4, 2 * (t % 4)] + acc[(t % 4) // GPB][t // 4 + 8, 2 * (t % 4) + 1]
+                     for t in range(32)])
+
+
+@pytest.mark.parametrize("fmt", ["int4", "fp4"])
+@pytest.mark.parametrize("G", [128, 64, 32])
+def test_set_of_blocks_gives_every_lane_a_row_group_dot_product(fmt, G):
+    rng = np.random.default_rng(300 + G + (0 if fmt == "int4" else 7))
+    GPB = 128 // G
+    S, RB = 4 // GPB, 16
+    NQ = RB // S
+    qs = {b: rng.integers(0, 16, size=(8, 128)) for b in range(RB)}
+    xs = {b: rng.standard_normal(128) for b in range(RB)}
+    scale = 2.0 ** -24 if fmt == "int4" else 1.0
+    covered = set()
+    for q in range(NQ):
+        lanes = emulate_set(fmt, qs, xs, G, q, NQ)
+        for t in range(32):
+            g, r = t // 4, t % 4
+            blk, h = q + NQ * (r // GPB), r % GPB
+            ks = range(h * G, (h + 1) * G)
+            dq = [qs[blk][g, k] * scale if fmt == "int4" else e2m1(int(qs[blk][g, k])) for k in ks]
+            want = float(np.dot(dq, xs[blk][list(ks)]))
+            assert lanes[t] == pytest.approx(want, rel=1e-12, abs=1e-30), (q, t)
+            covered.add((g, blk, h))
+    assert len(covered) == 8 * RB * GPB          # every (row, block, group) of the item exactly once

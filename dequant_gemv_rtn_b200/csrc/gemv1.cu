@@ -801,4 +801,44 @@ cudaError_t launch_gemv_seq(const qnt_seq_step* steps, int n, int xbf16, void* w
   return b1_dispatch<QNT_SEQ_MAX_STEPS>(steps, n, xbf16, static_cast<unsigned*>(work), st, s, true, handled);
 }
 
+// ------------------------------------------------------------------ the same, with a library-owned workspace
+// For callers that cannot allocate device memory (qnt_gemv_seq_noalloc): the
+// completion counters live in this array, which the CUDA runtime places in the
+// device memory of every GPU that loads the library, for the life of the
+// process.  Host code must not pass the array's name to a kernel (on the host
+// it is only a stand-in); its device address is looked up once per device.
+static __device__ __align__(256) unsigned g_seq_counters[QNT_SEQ_NOALLOC_MAX_STEPS + 1];
+
+// Device address of g_seq_counters on the current device, looked up on the
+// first call for each device.
+static cudaError_t seq_counters_address(unsigned** out) {
+  static unsigned* addr[64] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_seq_counters);
+    if (e != cudaSuccess) return e;
+    addr[dev] = static_cast<unsigned*>(p);
+  }
+  *out = addr[dev];
+  return cudaSuccess;
+}
+
+cudaError_t launch_gemv_seq_noalloc(const qnt_seq_step* steps, int n, int xbf16, int* st, cudaStream_t s,
+                                    bool* handled) {
+  *handled = false;
+  unsigned* counters = nullptr;
+  cudaError_t e = seq_counters_address(&counters);
+  if (e != cudaSuccess) return e;
+  // every call starts from zeroed counters (the array keeps the last call's)
+  e = cudaMemsetAsync(counters, 0, sizeof(unsigned) * (size_t)(n + 1), s);
+  if (e != cudaSuccess) return e;
+  return b1_dispatch<QNT_SEQ_MAX_STEPS>(steps, n, xbf16, counters, st, s, true, handled);
+}
+
 }  // namespace qnt

@@ -35,6 +35,11 @@ cudaError_t launch_gemv4_one(const qnt_desc& d, const void* codes, const void* m
 cudaError_t launch_gemv_seq(const qnt_seq_step* steps, int n, int xbf16, void* work, int* st, cudaStream_t s,
                             bool* handled);
 
+// qnt_gemv_seq with the completion counters in a library-owned device array
+// (gemv1.cu); n <= QNT_SEQ_NOALLOC_MAX_STEPS.
+cudaError_t launch_gemv_seq_noalloc(const qnt_seq_step* steps, int n, int xbf16, int* st, cudaStream_t s,
+                                    bool* handled);
+
 // An empty kernel: the next kernel in the stream cannot overlap the ones before it.
 cudaError_t launch_stream_fence(cudaStream_t s);
 

@@ -155,9 +155,43 @@ int qnt_quantize(const qnt_desc* desc, const float* d_W, void* d_codes, void* d_
   return cuda_rc(qnt::launch_stream_fence(s));
 }
 
+}  // extern "C"
+
+namespace {
+// Validation of the steps of qnt_gemv_seq_noalloc (the rules of qnt_gemv_seq).
+int check_seq(const qnt_seq_step* steps, int nsteps, int xdtype) {
+  if (xdtype != QNT_F16 && xdtype != QNT_BF16) return QNT_ERR_ARG;
+  for (int i = 0; i < nsteps; ++i) {
+    const qnt_seq_step& t = steps[i];
+    const int e = check(&t.desc);
+    if (e != QNT_OK) return e;
+    if (!is_4bit(t.desc.fmt) || t.desc.fmt != steps[0].desc.fmt || t.desc.group != steps[0].desc.group)
+      return QNT_ERR_ARG;
+    if (t.wait < 0 || t.wait > i) return QNT_ERR_ARG;
+    if (t.desc.K > QNT_MAX_GEMV_K) return QNT_ERR_SHAPE;
+    if (!t.codes || !t.meta || !t.x || !t.y) return QNT_ERR_ARG;
+    if (!aligned16(t.codes) || !aligned16(t.meta) || !aligned16(t.x) || !aligned16(t.y)) return QNT_ERR_ALIGN;
+  }
+  return QNT_OK;
+}
+}  // namespace
+
+extern "C" {
+
 size_t qnt_gemv_seq_work_bytes(int nsteps) {
   if (nsteps < 1 || nsteps > QNT_SEQ_MAX_STEPS) return 0;
   return (size_t)round_up(4L * (nsteps + 1), 16);   // a counter per step, then an abort word
+}
+
+int qnt_gemv_seq_noalloc(const qnt_seq_step* steps, int nsteps, int xdtype, int* d_status, void* stream) {
+  if (!steps || nsteps < 1 || nsteps > QNT_SEQ_NOALLOC_MAX_STEPS) return QNT_ERR_ARG;
+  const int v = check_seq(steps, nsteps, xdtype);
+  if (v != QNT_OK) return v;
+  bool handled = false;
+  const int rc = cuda_rc(qnt::launch_gemv_seq_noalloc(steps, nsteps, xdtype == QNT_BF16, d_status,
+                                                      static_cast<cudaStream_t>(stream), &handled));
+  if (rc != QNT_OK) return rc;
+  return handled ? QNT_OK : QNT_ERR_SHAPE;
 }
 
 int qnt_gemv_seq(const qnt_seq_step* steps, int nsteps, int xdtype, void* d_work, int* d_status, void* stream) {

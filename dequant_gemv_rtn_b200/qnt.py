@@ -24,6 +24,7 @@ FORMATS = {"int4": QNT_INT4_ASYM, "fp4": QNT_FP4_E2M1, "afpq": QNT_FP4_AFPQ, "ra
 
 QNT_MAX_GEMV_K = 65536
 QNT_SEQ_MAX_STEPS = 256
+QNT_SEQ_NOALLOC_MAX_STEPS = 256
 
 
 class qnt_desc(ctypes.Structure):
@@ -51,6 +52,7 @@ def _load():
         "qnt_gemm": (I, [D, P, P, P, P, I, I, P, P]),
         "qnt_gemv_seq_work_bytes": (Z, [I]),
         "qnt_gemv_seq": (I, [ctypes.POINTER(qnt_seq_step), I, I, P, P, P]),
+        "qnt_gemv_seq_noalloc": (I, [ctypes.POINTER(qnt_seq_step), I, I, P, P]),
         "qnt_table_create": (P, [I, I]),
         "qnt_table_set": (I, [P, ctypes.c_char_p, I, I]),
         "qnt_table_lookup": (I, [P, ctypes.c_char_p, ctypes.POINTER(I), ctypes.POINTER(I)]),
@@ -165,6 +167,12 @@ def qnt_gemv_seq(steps, xdtype: int, work, status=None, stream=None, check=True)
     """steps: a ctypes array from seq_steps() (host memory)."""
     rc = lib.qnt_gemv_seq(steps, len(steps), int(xdtype), _ptr(work), _ptr(status), _stream(stream))
     return _check(rc, "qnt_gemv_seq") if check else rc
+
+
+def qnt_gemv_seq_noalloc(steps, xdtype: int, status=None, stream=None, check=True) -> int:
+    """qnt_gemv_seq without a caller workspace (the library's own counters)."""
+    rc = lib.qnt_gemv_seq_noalloc(steps, len(steps), int(xdtype), _ptr(status), _stream(stream))
+    return _check(rc, "qnt_gemv_seq_noalloc") if check else rc
 
 
 class qnt_table:

@@ -254,6 +254,30 @@ size_t qnt_gemv_seq_work_bytes(int nsteps);
 int qnt_gemv_seq(const qnt_seq_step* steps, int nsteps, int xdtype, void* d_work, int* d_status, void* stream);
 
 /*
+ * qnt_gemv_seq_noalloc -- qnt_gemv_seq for callers that cannot allocate device
+ * memory: for example a host framework whose device memory is entirely handed
+ * out by its own pool, or a plug-in that is not allowed to call the CUDA
+ * allocator, and so cannot provide d_work.  It computes exactly what
+ * qnt_gemv_seq computes (same arguments, ordering, accuracy and errors) and
+ * allocates nothing.  (No counterpart in the pages: an interface convenience.)
+ *   Workspace: the per-step completion counters live in a small array that the
+ *     library itself places in the memory of every GPU that loads it, for the
+ *     life of the process ((QNT_SEQ_NOALLOC_MAX_STEPS + 1) * 4 bytes per GPU).
+ *     Each call clears the part it uses on `stream` before its kernel; the
+ *     array keeps the last call's contents afterwards.
+ *   Limit: nsteps <= QNT_SEQ_NOALLOC_MAX_STEPS, else QNT_ERR_ARG.
+ *   Every call shares the one array: two calls whose work overlaps on the GPU
+ *     (other streams, other host threads) race and may hang until their waits
+ *     expire (QNT_ERR_TIMEOUT); serialize them, or use qnt_gemv_seq with one
+ *     workspace each.
+ *   The first call on each device looks up the array's device address (a
+ *     runtime query, no allocation); make that first call before capturing a
+ *     stream into a CUDA graph.
+ */
+#define QNT_SEQ_NOALLOC_MAX_STEPS 256
+int qnt_gemv_seq_noalloc(const qnt_seq_step* steps, int nsteps, int xdtype, int* d_status, void* stream);
+
+/*
  * Selective precision (RTN page: raise the precision format of chosen layers
  * and modules).  A host-side table of ordered rules; qnt_table_lookup returns
  * the format and group of the first rule whose pattern matches the module name

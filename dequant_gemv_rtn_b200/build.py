@@ -16,6 +16,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OBJ = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libqnt.so")
+TEST_OBJ = os.path.join(PKG, "_build_test")
+TEST_LIB = os.path.join(PKG, "libqnt_test.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
@@ -32,16 +34,17 @@ def _deps():
     return _sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = None) -> bool:
+    lib = lib or LIB
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def _compile(src: str, verbose: bool, ptxas_v: bool) -> str:
-    obj = os.path.join(OBJ, os.path.basename(src) + ".o")
-    cmd = ["nvcc", *NVCC_FLAGS, "-c", src, "-o", obj]
+def _compile(src: str, verbose: bool, ptxas_v: bool, objdir: str = None, extra=()) -> str:
+    obj = os.path.join(objdir or OBJ, os.path.basename(src) + ".o")
+    cmd = ["nvcc", *NVCC_FLAGS, *extra, "-c", src, "-o", obj]
     if ptxas_v and src.endswith(".cu"):
         cmd.insert(1, "-Xptxas=-v")
     if verbose:
@@ -54,18 +57,25 @@ def _compile(src: str, verbose: bool, ptxas_v: bool) -> str:
     return obj
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_v: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(OBJ, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, ptxas_v: bool = False, test: bool = False) -> str:
+    """Build libqnt.so; with test=True the test library libqnt_test.so instead
+    (the same sources compiled with QNT_TEST_FAULTS: fault injection for the
+    tests of the bounded waits; the product library never contains it)."""
+    lib, obj, extra = (TEST_LIB, TEST_OBJ, ["-DQNT_TEST_FAULTS"]) if test else (LIB, OBJ, [])
+    if not force and up_to_date(lib):
+        return lib
+    os.makedirs(obj, exist_ok=True)
     with cf.ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose, ptxas_v), _sources()))
-    cmd = ["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", LIB, *objs, "-lcudart"]
+        objs = list(ex.map(lambda s: _compile(s, verbose, ptxas_v, obj, extra), _sources()))
+    cmd = ["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", lib, *objs, "-lcudart"]
+    if test:   # its own calls bind to its own definitions, even beside libqnt.so
+        cmd += ["-Xlinker", "-Bsymbolic"]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.check_call(cmd)
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, ptxas_v="--ptxas-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, ptxas_v="--ptxas-v" in sys.argv,
+                test="--test" in sys.argv))

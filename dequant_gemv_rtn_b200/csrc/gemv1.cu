@@ -84,7 +84,7 @@ struct B1Params {
   int kmax;
   int meta_cap;     // bytes of one staged metadata window
   int part_cap;     // floats of the per-row partial-sum table
-  int pad;
+  int fault;        // test builds only: an injected fault (0: none)
   unsigned* done;   // [nsteps] completion counters, then one abort word (sequence only)
   int* status;
   unsigned long long timeout_ns;
@@ -651,7 +651,13 @@ gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
       else reinterpret_cast<__half*>(st.y)[r_lo + rr] = __float2half_rn(v);
     }
     consumer_bar(nct);
-    if (P.done && tid == 0)   // release: every y store of the CTA (ordered by the barrier) comes first
+#ifdef QNT_TEST_FAULTS
+    // test builds: CTA 0 never reports step 0 complete, so every wait for it expires
+    const bool skip_signal = P.fault == 1 && j == 0 && blockIdx.x == 0;
+#else
+    constexpr bool skip_signal = false;
+#endif
+    if (P.done && tid == 0 && !skip_signal)   // release: every y store of the CTA (ordered by the barrier) comes first
       asm volatile("red.release.gpu.global.add.u32 [%0], 1;" :: "l"(P.done + j) : "memory");
     T0 += nitems;
   }
@@ -664,6 +670,22 @@ gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
 }
 
 // ------------------------------------------------------------------ launchers
+#ifdef QNT_TEST_FAULTS
+// Test builds only: a fault to inject into the next launches of this thread and
+// the wait limit to use (set by qnt_test_gemv_seq_fault).
+static thread_local int t_fault = 0;
+static thread_local unsigned long long t_timeout_ns = kB1TimeoutNs;
+void set_test_fault(int fault, unsigned long long timeout_ns) {
+  t_fault = fault;
+  t_timeout_ns = timeout_ns;
+}
+#define QNT_B1_FAULT t_fault
+#define QNT_B1_TIMEOUT t_timeout_ns
+#else
+#define QNT_B1_FAULT 0
+#define QNT_B1_TIMEOUT kB1TimeoutNs
+#endif
+
 namespace {
 
 // Shared-memory plan of a launch: the deepest per-warp ring that fits with the
@@ -739,7 +761,8 @@ cudaError_t b1_launch(const qnt_seq_step* steps, int n, int xbf16, unsigned* don
   P.part_cap = p.part_cap;
   P.done = done;
   P.status = st;
-  P.timeout_ns = kB1TimeoutNs;
+  P.fault = QNT_B1_FAULT;
+  P.timeout_ns = QNT_B1_TIMEOUT;
   *handled = true;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);

@@ -40,6 +40,12 @@ cudaError_t launch_gemv_seq(const qnt_seq_step* steps, int n, int xbf16, void* w
 cudaError_t launch_gemv_seq_noalloc(const qnt_seq_step* steps, int n, int xbf16, int* st, cudaStream_t s,
                                     bool* handled);
 
+#ifdef QNT_TEST_FAULTS
+// Test builds only (gemv1.cu): inject `fault` into this thread's next batch-1 /
+// sequence launches and use `timeout_ns` as their wait limit.
+void set_test_fault(int fault, unsigned long long timeout_ns);
+#endif
+
 // An empty kernel: the next kernel in the stream cannot overlap the ones before it.
 cudaError_t launch_stream_fence(cudaStream_t s);
 

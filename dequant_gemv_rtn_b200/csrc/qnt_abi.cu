@@ -243,3 +243,18 @@ int qnt_gemv(const qnt_desc* desc, const void* d_codes, const void* d_meta, cons
 }
 
 }  // extern "C"
+
+#ifdef QNT_TEST_FAULTS
+// Test builds only (libqnt_test.so, never the product library): qnt_gemv_seq
+// with a fault injected and a short wait limit, so that a test can watch a
+// bounded wait expire.  fault 1: CTA 0 never reports step 0 complete, so every
+// step that waits for step 0 gives up after timeout_ns and the kernel reports
+// QNT_ERR_TIMEOUT, drains its copies and returns.
+extern "C" int qnt_test_gemv_seq_fault(const qnt_seq_step* steps, int nsteps, int xdtype, void* d_work,
+                                       int* d_status, void* stream, int fault, unsigned long long timeout_ns) {
+  qnt::set_test_fault(fault, timeout_ns);
+  const int rc = qnt_gemv_seq(steps, nsteps, xdtype, d_work, d_status, stream);
+  qnt::set_test_fault(0, 2000000000ull);
+  return rc;
+}
+#endif

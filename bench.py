@@ -69,6 +69,31 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def measured_tensor_peak():
+    """bf16 dense TFLOP/s measured by a seconds-long cuBLAS loop (sustained)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops_sustained" in d:
+            return d["bf16_tflops_sustained"], "measured (sustained)"
+    return 1400.0, "fallback (sustained)"
+
+
+META_BYTES_PER_GROUP = {1: 2.5, 2: 2.0, 3: 4.0, 4: 2.25}   # INT4, FP4, AFPQ, RaZeR
+
+
+def algo_bytes(fmt, N, K, M, g=GROUP):
+    """Algorithmic bytes of one GEMV / GEMM: codes + metadata + activations + outputs."""
+    if fmt == 5:                      # INT8 per channel: a byte per weight, an fp16 scale per row
+        wbytes = N * K + 2 * N
+    elif fmt == 6:                    # FP16
+        wbytes = 2 * N * K
+    else:
+        wbytes = N * K // 2 + int(N * K // g * META_BYTES_PER_GROUP[fmt])
+    return wbytes + 2 * K * M + 2 * N * M
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -442,6 +467,157 @@ def run_reference(args, world, rank, local):
             "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+# ------------------------------------------------------------------ the other workloads
+def _time_graph(torch, stream, run, warmup, reps):
+    """Capture run(stream) in a CUDA graph, replay; per-replay ms (CUDA events)."""
+    with torch.cuda.stream(stream):
+        run(stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        run(torch.cuda.current_stream())
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    ev = []
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            ev.append((a, b))
+    torch.cuda.synchronize()
+    out = [a.elapsed_time(b) for a, b in ev]
+    del g
+    return out
+
+
+def _quantized(Q, torch, synth, fmt, N, K, g, seed, st):
+    d = Q.desc(fmt, N, K, g)
+    W = synth.llama_like_device(N, K, seed=seed)
+    codes = torch.empty(Q.qnt_codes_bytes(d), dtype=torch.uint8, device="cuda")
+    meta = torch.empty(max(16, Q.qnt_meta_bytes(d)), dtype=torch.uint8, device="cuda")
+    Q.qnt_quantize(d, W, codes, meta, st)
+    del W
+    return d, codes, meta
+
+
+def run_extra_configs(args):
+    """The pages' other workloads, each in the launch configuration its parity
+    test covers: FP4 / AFPQ / RaZeR on K=4096, N=14336 at batch 1 and 4; the
+    Llama-70B INT4 GEMMs at M = 1..128 with bf16 activations; the
+    selective-precision Llama-2-7B stack at batch 1 and 16.  Each matrix is
+    timed over enough rotating copies that its weights come from HBM."""
+    import torch
+    from dequant_gemv_rtn_b200 import qnt as Q
+    from dequant_gemv_rtn_b200 import synth
+    hbm, hbm_kind = measured_peaks()
+    tpeak, tkind = measured_tensor_peak()
+    stream = torch.cuda.Stream()
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pct = lambda v, q: float(np.percentile(v, q))
+    reps = 20
+    out = {"peaks": {"hbm_GBps": hbm, "hbm_kind": hbm_kind, "bf16_TFLOPs": tpeak, "bf16_kind": tkind}}
+
+    def timed(name, fmt, N, K, M, xdt, copies):
+        """copies: list of (d, codes, meta); times qnt_gemv (M = 1) or qnt_gemm."""
+        X = synth.activations_device(M, K, seed=11, dtype=torch.bfloat16 if xdt else torch.float16)
+        Y = torch.empty((M, N), dtype=X.dtype, device="cuda")
+
+        def run(s):
+            for d, c, m in copies:
+                if M == 1:
+                    Q.qnt_gemv(d, c, m, X, Y, xdt, st, s)
+                else:
+                    Q.qnt_gemm(d, c, m, X, Y, M, xdt, st, s)
+        ms = _time_graph(torch, stream, run, 3, reps)
+        us = [t * 1000.0 / len(copies) for t in ms]
+        med = statistics.median(us)
+        byts = algo_bytes(fmt, N, K, M)
+        r = {"us": round(med, 3), "p10_p90_us": [round(pct(us, 10), 3), round(pct(us, 90), 3)],
+             "GBps": round(byts / med / 1e3, 1), "frac_hbm": round(byts / med / 1e3 / hbm, 4)}
+        if M > 1:
+            tfl = 2.0 * M * N * K / med / 1e6
+            r["TFLOPs"] = round(tfl, 1)
+            r["frac_tensor"] = round(tfl / tpeak, 4)
+        assert int(st.item()) == 0, f"{name}: device status {int(st.item())}"
+        return r
+
+    def ncopies(nbytes):
+        return max(2, min(8, int(4 * 126e6 // max(nbytes, 1)) + 1))
+
+    # FP4 family, K=4096 N=14336, batch 1 and 4 (fp16 activations)
+    for fmt, fname in ((2, "fp4"), (3, "afpq"), (4, "razer")):
+        N, K = 14336, 4096
+        copies = [_quantized(Q, torch, synth, fmt, N, K, GROUP, 40 + i, st) for i in range(ncopies(algo_bytes(fmt, N, K, 1)))]
+        for M in (1, 4):
+            out[f"{fname}_g128_{K}x{N}_b{M}"] = timed(fname, fmt, N, K, M, 0, copies)
+        del copies
+        torch.cuda.empty_cache()
+    # Llama-70B INT4 g128, bf16 activations, M sweep
+    for N, K in ((10240, 8192), (28672, 8192), (8192, 28672)):
+        copies = [_quantized(Q, torch, synth, 1, N, K, GROUP, 60 + i, st) for i in range(ncopies(algo_bytes(1, N, K, 1)))]
+        for M in (1, 8, 16, 32, 64, 128):
+            out[f"int4_g128_{K}x{N}_bf16_M{M}"] = timed("llama70b", 1, N, K, M, 1, copies)
+        del copies
+        torch.cuda.empty_cache()
+    # selective-precision Llama-2-7B stack: INT4 g128, INT8 per channel for
+    # down_proj of layers 0, 1, 30, 31, FP16 lm_head; batch 1 and 16
+    t = Q.qnt_table_create(Q.QNT_INT4_ASYM, GROUP)
+    for layer in (0, 1, 30, 31):
+        t.set(f"layers.{layer}.mlp.down_proj", Q.QNT_INT8_PERCHAN, 0)
+    t.set("lm_head", Q.QNT_FP16, 0)
+    mods = []
+    for l in range(32):
+        mods += [(f"layers.{l}.self_attn.{p}", 4096, 4096) for p in ("q_proj", "k_proj", "v_proj", "o_proj")]
+        mods += [(f"layers.{l}.mlp.gate_proj", 11008, 4096), (f"layers.{l}.mlp.up_proj", 11008, 4096),
+                 (f"layers.{l}.mlp.down_proj", 4096, 11008)]
+    stack, stack_bytes = [], {1: 0, 16: 0}
+    for i, (name, N, K) in enumerate(mods):
+        fmt, g = t.lookup(name)
+        stack.append((fmt, N, K) + _quantized(Q, torch, synth, fmt, N, K, g if g else K, 900 + i, st))
+        for M in (1, 16):
+            stack_bytes[M] += algo_bytes(fmt, N, K, M)
+    head = _quantized(Q, torch, synth, Q.QNT_FP16, 32000, 4096, 4096, 899, st)
+    t.close()
+    for M in (1, 16):
+        Xs = {K: synth.activations_device(M, K, seed=K, dtype=torch.float16) for K in (4096, 11008)}
+        Ys = {N: torch.empty((M, N), dtype=torch.float16, device="cuda") for N in (4096, 11008, 32000)}
+
+        def run_stack(s, M=M, Xs=Xs, Ys=Ys):
+            for fmt, N, K, d, c, m in stack:
+                if M == 1:
+                    Q.qnt_gemv(d, c, m, Xs[K], Ys[N], 0, st, s)
+                else:
+                    Q.qnt_gemm(d, c, m, Xs[K], Ys[N], M, 0, st, s)
+
+        def run_head(s, M=M, Xs=Xs, Ys=Ys):
+            d, c, m = head
+            if M == 1:
+                Q.qnt_gemv(d, c, m, Xs[4096], Ys[32000], 0, st, s)
+            else:
+                Q.qnt_gemm(d, c, m, Xs[4096], Ys[32000], M, 0, st, s)
+        ms = _time_graph(torch, stream, run_stack, 3, 10)
+        med = statistics.median(ms)
+        out[f"selective_stack_b{M}"] = {
+            "us_per_token_step": round(med * 1000.0, 1), "us_per_layer": round(med * 1000.0 / 32, 2),
+            "p10_p90_ms": [round(pct(ms, 10), 4), round(pct(ms, 90), 4)],
+            "GBps": round(stack_bytes[M] / (med * 1e-3) / 1e9, 1),
+            "frac_hbm": round(stack_bytes[M] / (med * 1e-3) / 1e9 / hbm, 4),
+            "how": "224 modules (INT4 g128; INT8 per-channel down_proj in layers 0,1,30,31) as qnt_gemv / "
+                   "qnt_gemm launches in one CUDA graph"}
+        hm = _time_graph(torch, stream, run_head, 3, 20)
+        hmed = statistics.median(hm)
+        hb = algo_bytes(6, 32000, 4096, M)
+        out[f"lm_head_fp16_b{M}"] = {"us": round(hmed * 1000.0, 2), "GBps": round(hb / (hmed * 1e-3) / 1e9, 1),
+                                     "frac_hbm": round(hb / (hmed * 1e-3) / 1e9 / hbm, 4)}
+    assert int(st.item()) == 0
+    del stack, head
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_kernel_only(name: str, fmt_name: str, repeats: int = 5):
     """Small case for profilers.  A layer shape: one matrix of that shape,
     quantized once, then `repeats` qnt_gemv launches (M=1, fp16 x).  "layer":
@@ -489,6 +665,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--no-extras", action="store_true", help="skip the other workloads")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.kernel_only:
@@ -505,6 +682,10 @@ def main():
         return
     import torch
     result, _ = run_ours(args, world, rank, local)
+    if world == 1 and not args.no_extras:
+        del _
+        torch.cuda.empty_cache()
+        result["extra_configs"] = run_extra_configs(args)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(torch, args.cpu_budget)
     if rank == 0:

@@ -49,6 +49,11 @@ void set_test_fault(int fault, unsigned long long timeout_ns);
 // An empty kernel: the next kernel in the stream cannot overlap the ones before it.
 cudaError_t launch_stream_fence(cudaStream_t s);
 
+// Y[m] = W x[m] for 1 <= M <= 128 on the tensor cores in one pass over the
+// weights (gemm_tc.cu, 4-bit formats).  *handled = false when it does not apply.
+cudaError_t launch_gemm_tc(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
+                           int M, int xbf16, int* st, cudaStream_t s, bool* handled);
+
 // Y[m] = W x[m] for m < M on the tensor cores (gemv_tc.cu).  Returns with
 // *handled = false, launching nothing, when the tensor-core kernel does not
 // take this format / batch / shape.

@@ -45,14 +45,13 @@ int check(const qnt_desc* d) {
   return QNT_OK;
 }
 
-// Y[m] = W x[m], m < M.  Kernel choice (measured on B200 with L2-cold weights,
-// 14336 x 4096 and the Llama-7B decode shapes):
-//   one vector, 4-bit formats        -> batch-1 kernel (mma.sync tensor cores)
-//   INT4 2..8 vectors; FP4; AFPQ;
-//   RaZeR 2 vectors                  -> CUDA-core multi-vector kernel
-//   INT4 from 9, RaZeR from 3 vectors -> tensor-core kernel (tcgen05), in
-//                                       passes of 16 vectors above 16
-//   INT8, FP16; FP4 / AFPQ above 8    -> CUDA-core multi-vector kernel (passes of 8)
+// Y[m] = W x[m], m < M.  Kernel choice (measured on B200 with L2-cold weights):
+//   one vector, 4-bit formats         -> batch-1 kernel (mma.sync tensor cores)
+//   9..128 vectors, 4-bit formats     -> tcgen05 GEMM, one pass over the weights
+//   INT4, FP4, AFPQ 2..8 vectors;
+//   RaZeR 2 vectors                   -> CUDA-core multi-vector kernel
+//   RaZeR 3..8 vectors                -> tcgen05 kernel for up to 16 vectors
+//   INT8, FP16                        -> CUDA-core multi-vector kernel (passes of 8)
 // QNT_FORCE_SIMT=1 selects the CUDA-core multi-vector kernel everywhere and
 // QNT_FORCE_TC=1 the tensor-core kernel wherever it applies (used to test every
 // path on the same inputs).
@@ -68,6 +67,10 @@ cudaError_t dispatch_gemm(const qnt_desc& d, const void* codes, const void* meta
   cudaError_t e = cudaSuccess;
   if (force == 0 && M == 1) {
     e = qnt::launch_gemv4_one(d, codes, meta, z0, X, Y, xbf16, st, s, &handled);
+    if (handled || e != cudaSuccess) return e;
+  }
+  if (force == 0 && M >= 9) {   // 4-bit formats: one pass over the weights on tcgen05
+    e = qnt::launch_gemm_tc(d, codes, meta, z0, X, Y, M, xbf16, st, s, &handled);
     if (handled || e != cudaSuccess) return e;
   }
   const bool tc = force == 2 || (force == 0 && ((d.fmt == QNT_INT4_ASYM && M > 8) || (d.fmt == QNT_FP4_RAZER && M > 2)));

@@ -618,47 +618,89 @@ def run_extra_configs(args):
     return out
 
 
-def run_kernel_only(name: str, fmt_name: str, repeats: int = 5):
-    """Small case for profilers.  A layer shape: one matrix of that shape,
-    quantized once, then `repeats` qnt_gemv launches (M=1, fp16 x).  "layer":
-    one decode layer (its five GEMVs) as `repeats` qnt_gemv_seq launches."""
+def run_kernel_only(name: str, fmt_name: str, M: int = 16, repeats: int = 5):
+    """Small cases for profilers, each a few launches of one kernel:
+      a layer shape (qkv, o, gate, up, down): one matrix of that shape, quantized
+        once, then `repeats` qnt_gemv launches (batch 1, fp16 x);
+      "layer": one decode layer (its five GEMVs, with the bench's waits) as
+        `repeats` qnt_gemv_seq launches;
+      "gemm": the Llama-70B gate/up matrix (K=8192, N=28672, INT4 g128) times M
+        bf16 activation rows, `repeats` qnt_gemm launches;
+      "quantize": qnt_quantize of the Llama-7B gate matrix (11008 x 4096 fp32);
+      "int8_down": the INT8 per-channel down_proj (K=11008, N=4096), qnt_gemv;
+      "fp16_lm_head": the FP16 lm_head (K=4096, N=32000), qnt_gemv."""
     import torch
     from dequant_gemv_rtn_b200 import qnt as Q
     from dequant_gemv_rtn_b200 import synth
-    fmt = Q.FORMATS[fmt_name]
-    mats = []
-    for i, (n, N, K) in enumerate(SHAPES):
-        if name not in ("layer", n):
-            continue
-        d = Q.desc(fmt, N, K, GROUP)
-        W = synth.llama_like_device(N, K, seed=3 + i)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def quantized(fmt, N, K, g, seed):
+        d = Q.desc(fmt, N, K, g)
+        W = synth.llama_like_device(N, K, seed=seed)
         codes = torch.empty(Q.qnt_codes_bytes(d), dtype=torch.uint8, device="cuda")
         meta = torch.empty(max(16, Q.qnt_meta_bytes(d)), dtype=torch.uint8, device="cuda")
-        Q.qnt_quantize(d, W, codes, meta)
-        del W
+        Q.qnt_quantize(d, W, codes, meta, st)
+        return d, codes, meta
+
+    shapes = []
+    if name == "gemm":
+        d, codes, meta = quantized(Q.QNT_INT4_ASYM, 28672, 8192, GROUP, 3)
+        X = synth.activations_device(M, 8192, seed=5, dtype=torch.bfloat16)
+        Y = torch.empty((M, 28672), dtype=torch.bfloat16, device="cuda")
+        for _ in range(repeats):
+            Q.qnt_gemm(d, codes, meta, X, Y, M, Q.QNT_BF16, st)
+        shapes, outs = [[28672, 8192, M]], [Y]
+    elif name == "quantize":
+        d = Q.desc(Q.QNT_INT4_ASYM, INTER, HIDDEN, GROUP)
+        W = synth.llama_like_device(INTER, HIDDEN, seed=3)
+        codes = torch.empty(Q.qnt_codes_bytes(d), dtype=torch.uint8, device="cuda")
+        meta = torch.empty(Q.qnt_meta_bytes(d), dtype=torch.uint8, device="cuda")
+        for _ in range(repeats):
+            Q.qnt_quantize(d, W, codes, meta, st)
+        shapes, outs = [[INTER, HIDDEN]], []
+    elif name in ("int8_down", "fp16_lm_head"):
+        fmt, N, K = (Q.QNT_INT8_PERCHAN, HIDDEN, INTER) if name == "int8_down" else (Q.QNT_FP16, 32000, HIDDEN)
+        d, codes, meta = quantized(fmt, N, K, K, 3)
         x = synth.activations_device(1, K, seed=5, dtype=torch.float16)
         y = torch.empty(N, dtype=torch.float16, device="cuda")
-        mats.append((d, codes, meta, x, y))
-    if name == "layer":
-        steps = Q.seq_steps([(d, c, m, x, y, 1 if i else 0) for i, (d, c, m, x, y) in enumerate(mats)])
-        work = torch.zeros(Q.qnt_gemv_seq_work_bytes(len(steps)), dtype=torch.uint8, device="cuda")
         for _ in range(repeats):
-            Q.qnt_gemv_seq(steps, Q.QNT_F16, work)
+            Q.qnt_gemv(d, codes, meta, x, y, Q.QNT_F16, st)
+        shapes, outs = [[N, K]], [y]
     else:
-        d, codes, meta, x, y = mats[0]
-        for _ in range(repeats):
-            Q.qnt_gemv(d, codes, meta, x, y, Q.QNT_F16)
+        fmt = Q.FORMATS[fmt_name]
+        layer_wait = {"qkv": 0, "o": 1, "gate": 1, "up": 2, "down": 1}
+        mats = []
+        for i, (n, N, K) in enumerate(SHAPES):
+            if name not in ("layer", n):
+                continue
+            d, codes, meta = quantized(fmt, N, K, GROUP, 3 + i)
+            x = synth.activations_device(1, K, seed=5, dtype=torch.float16)
+            y = torch.empty(N, dtype=torch.float16, device="cuda")
+            mats.append((n, d, codes, meta, x, y))
+        if name == "layer":
+            steps = Q.seq_steps([(d, c, m, x, y, layer_wait[n]) for n, d, c, m, x, y in mats])
+            work = torch.zeros(Q.qnt_gemv_seq_work_bytes(len(steps)), dtype=torch.uint8, device="cuda")
+            for _ in range(repeats):
+                Q.qnt_gemv_seq(steps, Q.QNT_F16, work, st)
+        else:
+            _, d, codes, meta, x, y = mats[0]
+            for _ in range(repeats):
+                Q.qnt_gemv(d, codes, meta, x, y, Q.QNT_F16, st)
+        shapes, outs = [[d.N, d.K] for _, d, *_ in mats], [m[5] for m in mats]
     torch.cuda.synchronize()
-    print(json.dumps({"kernel_only": name, "fmt": fmt_name, "launches": repeats,
-                      "shapes": [[d.N, d.K] for d, *_ in mats],
-                      "y_finite": all(bool(torch.isfinite(m[4].float()).all()) for m in mats)}))
+    assert int(st.item()) == 0, f"device status {int(st.item())}"
+    print(json.dumps({"kernel_only": name, "fmt": fmt_name, "launches": repeats, "shapes": shapes,
+                      "y_finite": all(bool(torch.isfinite(o.float()).all()) for o in outs)}))
 
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kernel-only", choices=[n for n, _, _ in SHAPES] + ["layer"], default=None,
-                    help="profiling case: one matrix of this shape (or one decode layer), a few launches")
-    ap.add_argument("--fmt", default="int4", help="format for --kernel-only")
+    ap.add_argument("--kernel-only", default=None,
+                    choices=[n for n, _, _ in SHAPES] + ["layer", "gemm", "quantize", "int8_down", "fp16_lm_head"],
+                    help="profiling case: a few launches of one kernel (see run_kernel_only)")
+    ap.add_argument("--fmt", default="int4", help="format for --kernel-only with a layer shape")
+    ap.add_argument("--m", type=int, default=16, help="activation rows for --kernel-only gemm")
+    ap.add_argument("--repeats", type=int, default=5, help="launches for --kernel-only")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
@@ -669,7 +711,7 @@ def main():
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.kernel_only:
-        run_kernel_only(args.kernel_only, args.fmt)
+        run_kernel_only(args.kernel_only, args.fmt, args.m, args.repeats)
         return
     world, rank, local = dist_setup(args.gpus)
     if args.impl == "reference":

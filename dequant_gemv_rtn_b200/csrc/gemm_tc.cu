@@ -1,5 +1,5 @@
 // gemm_tc.cu -- small-batch fused-dequant GEMM on the 5th-generation tensor
-// cores (tcgen05), in one pass over the weights for 9 <= M <= 128 activation
+// cores (tcgen05), in one pass over the weights for 3 <= M <= 128 activation
 // rows: Y[m][n] = sum_k dq(code[n][k], meta[n][k/g]) * X[m][k].
 //
 // The GEMM of the RTN page ("Is (Selective) Round-To-Nearest Quantization All
@@ -10,23 +10,32 @@
 //
 // Structure: one CTA per tile of 128 weight rows (tensor-memory lanes), the
 // whole of K in stages of 128 weights:
-//  * warp 0 requests each stage: the stage's 512-byte block of each of the
-//    tile's 16 row groups (1-D bulk copies, one per lane) and the stage's slice
-//    of X as two 64-column boxes of a tensor map with 128-byte swizzle (rows of
-//    X beyond M read as zeros), so X is the canonical K-major B operand;
-//  * warps 2..9 decode: each thread owns one weight row (its tensor-memory
-//    lane) and half of the stage's 128 weights, turns the codes into the MMA's
-//    A operand with the group scale folded in (one rounding per weight: fp16
-//    (q - z) exactly, times the scale times a per-row power of two that keeps
-//    the products in fp16 range; bf16 the same product rounded once, through a
-//    split of the scale into bf16 high and low parts), and writes it to tensor
-//    memory with tcgen05.st;
-//  * warp 1 allocates tensor memory and one thread issues, per stage, eight
-//    tcgen05.mma (M = 128, N = M rounded up to 16, K = 16; A from tensor memory,
-//    B from shared memory; fp32 accumulation in tensor memory), committed to the
-//    stage's barrier, which frees its shared memory and its A columns;
-//  * the decode warps then read the accumulators (tcgen05.ld), undo the row's
+//  * warp 0 requests each stage with two kinds of TMA tile copies: the
+//    stage's 512-byte block of each of the tile's 16 row groups as one box of a
+//    2-D tensor map over the codes (row groups x 32-bit words), and the stage's
+//    slice of X as two 64-column boxes of a tensor map with 128-byte swizzle
+//    (rows of X beyond M read as zeros), so X is the canonical K-major B
+//    operand.  The shared-memory ring holds up to 16 stages;
+//  * the decode warps, in groups of four (one per tensor-memory lane quarter),
+//    take the stages in turn (group j: stages j, j + groups, ...): each thread
+//    owns one weight row (its tensor-memory lane) and turns the stage's 128
+//    weights of it into the MMA's A operand with the group scale folded in (one
+//    rounding per weight: fp16 (q - z) exactly, times the scale times a per-row
+//    power of two that keeps the products in fp16 range; bf16 the same product
+//    rounded once, through a split of the scale into bf16 high and low parts),
+//    and writes it to one of the A slots in tensor memory (the 64-column slots
+//    the accumulators leave, 4 or 6) with tcgen05.st;
+//  * one thread in each of warps 1..4 (2 or 4 of them, by M) issues a share of
+//    each stage's eight tcgen05.mma (M = 128, N = M rounded up to 16, K = 16;
+//    A from tensor memory, B from shared memory) into its own fp32
+//    accumulator in tensor memory, and commits them to the stage's barriers,
+//    which free the stage's shared memory and its A slot.  A single issuing
+//    thread is not enough: each small-N MMA occupies it for ~60 cycles, longer
+//    than the HBM time of the 2048 weights it consumes;
+//  * the decode warps then sum the accumulators (tcgen05.ld), undo the row's
 //    power of two and store Y.
+// Waiting threads sleep between tries (nanosleep backoff), so the waiting warps
+// take few issue slots from the decode warps.
 // Programmatic dependent launch: the codes of the first stages are requested
 // before griddepcontrol.wait, X after it.  Every wait is bounded; on expiry the
 // kernel reports QNT_ERR_TIMEOUT, lets every copy and MMA it issued finish,
@@ -43,23 +52,33 @@ namespace {
 constexpr int kGtRows = 128;            // weight rows per tile (tensor-memory lanes)
 constexpr int kGtStageK = 128;          // weights of each row per stage (one block)
 constexpr int kGtCodeBytes = 16 * 512;  // codes of one stage: 16 row groups x one block
-constexpr int kGtThreads = 320;         // 10 warps
-constexpr int kGtDecodeWarp0 = 2;
-constexpr int kGtMaxStages = 6;
-constexpr uint32_t kGtTmemCols = 512;   // D: columns 0..127; A slots from column 128, 64 each
-constexpr uint32_t kGtColA = 128;
+constexpr int kGtMmaWarp0 = 1;          // warps 1..4: MMA issuers
+constexpr int kGtMaxIssuers = 4;
+constexpr int kGtDecodeWarp0 = 5;       // then the decode warps, in groups of four (one per lane quarter)
+#ifndef QNT_GT_DECODE_GROUPS
+#define QNT_GT_DECODE_GROUPS 2
+#endif
+constexpr int kGtGroups = QNT_GT_DECODE_GROUPS;   // decode groups: group j decodes stages j, j + kGtGroups, ...
+constexpr int kGtThreads = 32 * (kGtDecodeWarp0 + 4 * kGtGroups);
+constexpr int kGtMaxStages = 16;        // shared-memory ring
+constexpr int kGtMaxASlots = 8;         // A slots in tensor memory, at most
+constexpr uint32_t kGtTmemCols = 512;   // accumulators first, then the A slots, 64 columns each
 constexpr int kGtCtrl = 1024;
 constexpr unsigned long long kGtTimeoutNs = 2000000000ull;
 
 struct GtArgs {
-  const uint8_t* codes;
   const uint8_t* meta;
   void* Y;
   long z0;
   int N, K, M, Mpad;
-  int nstages;        // stages in flight (shared-memory and A slots)
+  int nstages;        // shared-memory stages in flight
+  int nissuers;       // MMA issuing threads (accumulators): 4 for M <= 64, else 2
+  int naslots;        // A slots: the tensor-memory columns the accumulators leave, 64 each, at most 8
+  int cola;           // first column of the A slots
   int xbf16;
   int* status;
+  unsigned long long timeout_ns;   // limit of every wait
+  int fault;                       // test builds only: an injected fault (0: none)
 };
 
 struct GtSmem { size_t stage0, stage_bytes, xoff, total; };
@@ -78,22 +97,52 @@ __device__ __forceinline__ uint64_t gt_now() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-// Bounded wait (gives up `timeout` ns after the first unsuccessful try or when
-// the abort flag is raised).
-__device__ __forceinline__ bool gt_wait(uint64_t* bar, uint32_t parity, volatile int* abort_s) {
+// Bounded wait (gives up `timeout` ns after the first unsuccessful try, or
+// when the abort flag is raised).  max_sleep > 0: between tries the thread
+// sleeps, 32 ns at first, doubling up to max_sleep ns, so a waiting warp takes
+// few issue slots from the decode warps that share its scheduler and sees the
+// phase complete at most ~max_sleep ns late.  max_sleep = 0: it spins, looking
+// at the flag and the clock every 64 tries (the MMA issuers, whose waits are on
+// the critical path).  (A suspend-time hint on try_wait instead was measured to
+// wake the thread up to microseconds after the phase completed.)
+__device__ __forceinline__ bool gt_wait(uint64_t* bar, uint32_t parity, volatile int* abort_s, uint64_t timeout,
+                                        uint32_t max_sleep) {
   const uint32_t a = smem_addr(bar);
   uint64_t deadline = 0;
-  for (;;) {
+  for (uint32_t n = 0, ns = 0;; ++n) {
     uint32_t done;
     asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
                  : "=r"(done) : "r"(a), "r"(parity) : "memory");
     if (done) return true;
+    if (max_sleep == 0 && (n & 63u) != 63u) continue;
     if (abort_s && *abort_s) return false;
     const uint64_t now = gt_now();
-    if (deadline == 0) deadline = now + kGtTimeoutNs;
+    if (deadline == 0) deadline = now + timeout;
     else if (now > deadline) return false;
+    if (max_sleep) {
+      if (ns) __nanosleep(ns);
+      ns = ns ? (ns < max_sleep ? 2 * ns : max_sleep) : 32;
+    }
   }
 }
+// Position in a ring of n slots: slot index and the parity of its current use.
+struct GtRing {
+  int slot = 0;
+  uint32_t phase = 0;
+  __device__ __forceinline__ void next(int n) {
+    if (++slot == n) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+  __device__ __forceinline__ void adv(int k, int n) {   // k <= n
+    slot += k;
+    if (slot >= n) {
+      slot -= n;
+      phase ^= 1u;
+    }
+  }
+};
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
@@ -136,11 +185,19 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 __device__ __forceinline__ uint32_t f16_idesc(int n, int bf16) {
   return (1u << 4) | (bf16 ? ((1u << 7) | (1u << 10)) : 0u) | ((uint32_t)(n >> 3) << 17) | ((128u >> 4) << 24);
 }
-// 2-D tiled TMA load (no multicast) of a box at (c0, c1) into shared memory.
+// 2-D tiled TMA loads (no multicast) of a box at (c0, c1) into shared memory.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
       :: "r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_addr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar,
+                                                 uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;"
+      :: "r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_addr(bar)), "l"(pol)
       : "memory");
 }
 
@@ -246,7 +303,7 @@ __device__ __forceinline__ GtGroup gt_group(uint32_t raw, float pw) {
 template <int FMT, bool BF16>
 __device__ __forceinline__ void gt_decode_chunk(const uint4& cv, const GtGroup& c, uint32_t (&a)[16]) {
   const uint32_t w[4] = {cv.x, cv.y, cv.z, cv.w};
-  if (FMT == QNT_INT4_ASYM) {
+  if constexpr (FMT == QNT_INT4_ASYM) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       // nibbles p = 0..7 of word j: chunk weights 16(p%2) + 4j + 2((p/2)%2) + p/4
@@ -268,8 +325,7 @@ __device__ __forceinline__ void gt_decode_chunk(const uint4& cv, const GtGroup& 
         a[8 + 2 * j + 1] = hmul2_(hsub2(and_or(w8, 0x00F000F0u, 0x64006400u), c.zhi), c.s2);
       }
     }
-    return;
-  }
+  } else {
   // FP4 family: byte b of word j holds chunk weights 8j + 2b, 8j + 2b + 1
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -303,40 +359,45 @@ __device__ __forceinline__ void gt_decode_chunk(const uint4& cv, const GtGroup& 
       }
     }
   }
+  }
 }
 
 // ------------------------------------------------------------------ kernel
 template <int FMT, int G, bool BF16>
 __global__ void __launch_bounds__(kGtThreads, 1)
-gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const GtArgs A) {
+gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap cmap, const GtArgs A) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);       // [nst] codes + X landed
-  uint64_t* afull = full + kGtMaxStages;                     // [nst] A written to tensor memory
-  uint64_t* empty = afull + kGtMaxStages;                    // [nst] the stage's MMAs are complete
-  uint64_t* dfull = empty + kGtMaxStages;                    // all MMAs complete
+  uint64_t* empty = full + kGtMaxStages;                     // [nst] the stage's MMAs are complete
+  uint64_t* afull = empty + kGtMaxStages;                    // [A slots] A written to tensor memory
+  uint64_t* aempty = afull + kGtMaxASlots;                   // [A slots] the MMAs reading the slot are complete
+  uint64_t* dfull = aempty + kGtMaxASlots;                   // all MMAs complete
   uint64_t* tmem_ready = dfull + 1;
   uint32_t* tbase_p = reinterpret_cast<uint32_t*>(smem + 512);
   volatile int* abort_s = reinterpret_cast<volatile int*>(smem + 520);
-  const int nst = A.nstages;
+  const int nst = A.nstages, nI = A.nissuers, nA = A.naslots;
   const GtSmem L = gt_smem(A.Mpad, nst);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int KB = A.K / 128, GK = A.K / G, NG = (A.N + 7) / 8;
+  const int KB = A.K / 128, GK = A.K / G;
   const int tile = blockIdx.x;
 
   if (tid == 0) {
     for (int i = 0; i < nst; ++i) {
       mbar_init_nofence(full + i, 1);
-      mbar_init_nofence(afull + i, 8);
-      mbar_init_nofence(empty + i, 1);
+      mbar_init_nofence(empty + i, nI);
     }
-    mbar_init_nofence(dfull, 1);
+    for (int i = 0; i < nA; ++i) {
+      mbar_init_nofence(afull + i, 4);
+      mbar_init_nofence(aempty + i, nI);
+    }
+    mbar_init_nofence(dfull, nI);
     mbar_init_nofence(tmem_ready, 1);
     mbar_init_fence();
     *abort_s = 0;
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   }
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kGtMmaWarp0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                  :: "r"(smem_addr(tbase_p)), "r"(kGtTmemCols) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -348,88 +409,84 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const GtArgs A) {
     *abort_s = 1;
     report(A.status, QNT_ERR_TIMEOUT);
   };
+  auto wait = [&](uint64_t* bar, uint32_t parity, volatile int* ab, uint32_t max_sleep = 128) {
+    return gt_wait(bar, parity, ab, A.timeout_ns, max_sleep);
+  };
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
-    const uint64_t pol = l2_evict_first_policy();
-    const int ng_tile = min(16, NG - tile * 16);               // row groups of the tile in the buffer
-    const uint32_t stage_tx = (uint32_t)ng_tile * 512u + (uint32_t)A.Mpad * 256u;
-    auto issue_codes = [&](int s) {
-      const int slot = s % nst;
-      uint8_t* st = smem + L.stage0 + (size_t)slot * L.stage_bytes;
-      if (lane == 0) mbar_expect_tx(full + slot, stage_tx);   // codes and X of the stage
-      __syncwarp();
-      if (lane < ng_tile)
-        bulk_g2s_hint(st + lane * 512, A.codes + (long)(tile * 16 + lane) * 4L * A.K + (long)s * 512, 512u,
-                      full + slot, pol);
-    };
-    auto issue_x = [&](int s) {
-      const int slot = s % nst;
-      uint8_t* st = smem + L.stage0 + (size_t)slot * L.stage_bytes;
-      if (lane == 0) {
-        tma_load_2d(st + L.xoff, &xmap, s * kGtStageK, 0, full + slot);
-        tma_load_2d(st + L.xoff + (size_t)A.Mpad * 128, &xmap, s * kGtStageK + 64, 0, full + slot);
-      }
-    };
-    // the first stages' codes do not depend on the preceding kernel; X does
-    const int pre = min(nst, KB);
-    int s = 0;
-    bool ok = true;
-    for (; s < pre; ++s) issue_codes(s);
-    if (lane == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
-    __syncwarp();
-    for (int i = 0; i < pre; ++i) issue_x(i);
-    for (; s < KB && ok; ++s) {
-      const int slot = s % nst;
-      if (lane == 0) ok = gt_wait(empty + slot, (uint32_t)(s / nst - 1) & 1u, abort_s);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) {
-        if (lane == 0 && !*abort_s) fail();
-        break;
-      }
-      issue_codes(s);
-      issue_x(s);
-    }
-    // drain: the copies of every issued stage have landed
-    if (lane == 0)
-      for (int i = (s > nst ? s - nst : 0); i < s; ++i) gt_wait(full + i % nst, (uint32_t)(i / nst) & 1u, nullptr);
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      int issued = 0;   // stages whose MMAs were issued and committed
-      if (!gt_wait(tmem_ready, 0, abort_s)) {
+      const uint64_t pol = l2_evict_first_policy();
+      const uint32_t stage_tx = (uint32_t)kGtCodeBytes + (uint32_t)A.Mpad * 256u;   // full boxes, zero-filled past the ends
+      auto stage_ptr = [&](int s) { return smem + L.stage0 + (size_t)(s % nst) * L.stage_bytes; };
+      auto issue_codes = [&](int s) {
+        mbar_expect_tx(full + s % nst, stage_tx);
+        tma_load_2d_hint(stage_ptr(s), &cmap, s * 128, tile * 16, full + s % nst, pol);
+      };
+      auto issue_x = [&](int s) {
+        uint8_t* st = stage_ptr(s);
+        tma_load_2d(st + L.xoff, &xmap, s * kGtStageK, 0, full + s % nst);
+        tma_load_2d(st + L.xoff + (size_t)A.Mpad * 128, &xmap, s * kGtStageK + 64, 0, full + s % nst);
+      };
+      // the first stages' codes do not depend on the preceding kernel; X does
+      const int pre = min(nst, KB);
+      int s = 0;
+      for (; s < pre; ++s) issue_codes(s);
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      for (int i = 0; i < pre; ++i) issue_x(i);
+      GtRing er;   // the stage whose slot stage s reuses: s - nst
+      for (; s < KB; ++s) {
+        if (!wait(empty + er.slot, er.phase, abort_s, 512)) {
+          if (!*abort_s) fail();
+          break;
+        }
+        er.next(nst);
+        issue_codes(s);
+        issue_x(s);
+      }
+      // drain: the copies of every issued stage have landed
+      for (int i = (s > nst ? s - nst : 0); i < s; ++i) wait(full + i % nst, (uint32_t)(i / nst) & 1u, nullptr);
+    }
+  } else if (warp < kGtMmaWarp0 + kGtMaxIssuers) {
+    // ---------------------------------------------------------------- MMA issuers
+    const int me = warp - kGtMmaWarp0;
+    if (lane == 0 && me < nI) {
+      if (!wait(tmem_ready, 0, abort_s)) {
         if (!*abort_s) fail();
       } else {
         tc_fence_after();
         const uint32_t tbase = *tbase_p;
+        const uint32_t dcol = tbase + (uint32_t)(me * A.Mpad);
         const uint32_t idesc = f16_idesc(A.Mpad, BF16 ? 1 : 0);
         const uint32_t st0 = smem_addr(smem + L.stage0);
+        const int per = 8 / nI, kk0 = me * per;
+        GtRing fr, ar;
         for (int s = 0; s < KB; ++s) {
-          const int slot = s % nst;
-          const uint32_t par = (uint32_t)(s / nst) & 1u;
-          if (!gt_wait(full + slot, par, abort_s) || !gt_wait(afull + slot, par, abort_s)) {
+          const int slot = fr.slot, as = ar.slot;
+          if (!wait(full + slot, fr.phase, abort_s, 0) || !wait(afull + as, ar.phase, abort_s, 0)) {
             if (!*abort_s) fail();
             break;
           }
+          fr.next(nst);
+          ar.next(nA);
           tc_fence_after();
           const uint32_t xs = st0 + (uint32_t)(slot * L.stage_bytes + L.xoff);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t acol = tbase + (uint32_t)A.cola + 64u * (uint32_t)as;
+          for (int kk = kk0; kk < kk0 + per; ++kk) {
             const uint32_t b_addr = xs + (uint32_t)((kk >> 2) * A.Mpad * 128) + 32u * (uint32_t)(kk & 3);
-            tc_mma_tmem_a(tbase, tbase + kGtColA + 64u * (uint32_t)slot + 8u * (uint32_t)kk, sw128_desc(b_addr),
-                          idesc, (s > 0 || kk > 0) ? 1u : 0u);
+            tc_mma_tmem_a(dcol, acol + 8u * (uint32_t)kk, sw128_desc(b_addr), idesc, (s > 0 || kk > kk0) ? 1u : 0u);
           }
           tc_commit(empty + slot);
-          ++issued;
+          tc_commit(aempty + as);
         }
-        tc_commit(dfull);   // arrives once every MMA issued above has completed
       }
+      tc_commit(dfull);   // arrives once every MMA this thread issued has completed
     }
-  } else if (warp >= kGtDecodeWarp0) {
+  } else {
     // ---------------------------------------------------------------- decode and epilogue
-    const int dw = warp - kGtDecodeWarp0;                      // 0..7
+    const int dw = warp - kGtDecodeWarp0;
     const int quarter = warp & 3;                              // tensor-memory lanes 32 quarter ..
-    const int half = dw >> 2;                                  // chunks 2 half, 2 half + 1
+    const int grp = dw >> 2;                                   // stages grp, grp + kGtGroups, ...
     const int r = 32 * quarter + lane;                         // row of the tile
     const long row = (long)tile * kGtRows + r;
     const bool rowok = row < A.N;
@@ -457,7 +514,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const GtArgs A) {
       unpw = __uint_as_float((uint32_t)(127 - e) << 23);
     }
     uint32_t tbase = 0;
-    bool ok = gt_wait(tmem_ready, 0, abort_s);
+    bool ok = wait(tmem_ready, 0, abort_s);
     if (ok) {
       tc_fence_after();
       tbase = *tbase_p;
@@ -466,62 +523,85 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const GtArgs A) {
     }
     const uint32_t tlane = (uint32_t)(32 * quarter) << 16;
     const uint32_t st0 = smem_addr(smem + L.stage0);
-    // raw metadata of this half's two chunks, requested kPf stages ahead
-    constexpr int kPf = 4;
-    uint32_t raw[kPf][2];
-    auto load_raw = [&](int s, uint32_t (&out)[2]) {
+    // raw metadata of the row's groups in a stage, requested kPf of this
+    // group's stages ahead
+    constexpr int kGps = 128 / G;   // groups per stage
+    constexpr int kPf = 2;
+    uint32_t raw[kPf][kGps];
+    auto load_raw = [&](int s, uint32_t (&out)[kGps]) {
       if (s >= KB) return;
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
-        out[h] = gt_meta_raw<FMT>(A.meta, A.z0, rowm * GK + ((long)s * 128 + (2 * half + h) * 32) / G);
+      for (int h = 0; h < kGps; ++h) out[h] = gt_meta_raw<FMT>(A.meta, A.z0, rowm * GK + (long)s * kGps + h);
     };
 #pragma unroll
-    for (int u = 0; u < kPf; ++u) load_raw(u, raw[u]);
-    for (int s0 = 0; s0 < KB && ok; s0 += kPf) {
+    for (int u = 0; u < kPf; ++u) load_raw(grp + u * kGtGroups, raw[u]);
+    // ring positions of this group's next stage; nst and nA are multiples of
+    // kGtGroups, so the stage that last used a slot was this group's own
+    GtRing fr, ar;
+    fr.adv(grp, nst);
+    ar.adv(grp, nA);
+    for (int s0 = grp; s0 < KB && ok; s0 += kGtGroups * kPf) {
 #pragma unroll
       for (int u = 0; u < kPf; ++u) {
-        const int s = s0 + u;
+        const int s = s0 + u * kGtGroups;
         if (s >= KB || !ok) break;
-        const int slot = s % nst;
-        GtGroup c[2];
+        GtGroup c[kGps];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) c[h] = gt_group<FMT, BF16>(raw[u][h], pw);
-        load_raw(s + kPf, raw[u]);
-        if (!gt_wait(full + slot, (uint32_t)(s / nst) & 1u, abort_s)) {
+        for (int h = 0; h < kGps; ++h) c[h] = gt_group<FMT, BF16>(raw[u][h], pw);
+        load_raw(s + kGtGroups * kPf, raw[u]);
+        const int slot = fr.slot, as = ar.slot;
+        if ((s >= nA && !wait(aempty + as, ar.phase ^ 1u, abort_s)) || !wait(full + slot, fr.phase, abort_s)) {
           if (!*abort_s) fail();
           ok = false;
           break;
         }
+        fr.adv(kGtGroups, nst);
+        ar.adv(kGtGroups, nA);
+        tc_fence_after();
         const uint32_t cbase = st0 + (uint32_t)(slot * L.stage_bytes) + (uint32_t)(rg * 512 + 64 * i8);
+        const uint32_t abase = tbase + tlane + (uint32_t)A.cola + 64u * (uint32_t)as;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int chunk = 2 * half + h;
+        for (int chunk = 0; chunk < 4; ++chunk) {
           const uint4 cv = lds128a(cbase + 16u * (uint32_t)(chunk ^ ((i8 >> 1) & 3)));
           uint32_t av[16];
-          gt_decode_chunk<FMT, BF16>(cv, c[h], av);
-          tmem_st16(tbase + tlane + kGtColA + 64u * (uint32_t)slot + 16u * (uint32_t)chunk, av);
+          gt_decode_chunk<FMT, BF16>(cv, c[chunk * 32 / G], av);
+          tmem_st16(abase + 16u * (uint32_t)chunk, av);
         }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0)
-          asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_addr(afull + slot)) : "memory");
+#ifdef QNT_TEST_FAULTS
+        // fault 1 (test builds): in CTA 0 the warp of lane quarter 0 never reports
+        // stage 0 decoded, so the MMA issuers' wait for it expires
+        const bool skip = A.fault == 1 && tile == 0 && s == 0 && quarter == 0;
+#else
+        constexpr bool skip = false;
+#endif
+        if (lane == 0 && !skip)
+          asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_addr(afull + as)) : "memory");
       }
     }
-    // epilogue: this half's columns of the accumulator rows
-    if (ok && gt_wait(dfull, 0, abort_s)) {
+    // epilogue: 16-column chunks of the accumulator rows, dealt out to the
+    // groups, summed over the accumulators
+    if (ok && wait(dfull, 0, abort_s)) {
       tc_fence_after();
-      // 16-column chunks of the accumulator rows, alternating between the halves
-      for (int cc = 16 * half; cc < A.Mpad; cc += 32) {
-        uint32_t d[16];
-        tmem_ld16(tbase + tlane + (uint32_t)cc, d);
-        tmem_wait_ld();
+      for (int cc = 16 * grp; cc < A.Mpad; cc += 16 * kGtGroups) {
+        float acc[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) acc[e] = 0.0f;
+        for (int i = 0; i < nI; ++i) {
+          uint32_t d[16];
+          tmem_ld16(tbase + tlane + (uint32_t)(i * A.Mpad + cc), d);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) acc[e] += __uint_as_float(d[e]);
+        }
         if (rowok) {
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int m = cc + e;
             if (m < A.M) {
-              const float v = __uint_as_float(d[e]) * unpw;
+              const float v = acc[e] * unpw;
               const size_t o = (size_t)m * A.N + row;
               if (A.xbf16) reinterpret_cast<__nv_bfloat16*>(A.Y)[o] = __float2bfloat16_rn(v);
               else reinterpret_cast<__half*>(A.Y)[o] = __float2half_rn(v);
@@ -535,8 +615,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const GtArgs A) {
   }
   // teardown: every MMA issued has completed before tensor memory is freed
   __syncthreads();
-  if (warp == 1) {
-    if (lane == 0 && *abort_s) gt_wait(dfull, 0, nullptr);   // the final commit follows every issued MMA
+  if (warp == kGtMmaWarp0) {
+    if (lane == 0 && *abort_s) wait(dfull, 0, nullptr);   // each issuer's final commit follows its MMAs
     __syncwarp();
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(*tbase_p), "r"(kGtTmemCols) : "memory");
@@ -544,6 +624,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const GtArgs A) {
 }
 
 // ------------------------------------------------------------------ host
+#ifdef QNT_TEST_FAULTS
+static thread_local int t_gt_fault = 0;
+static thread_local unsigned long long t_gt_timeout_ns = kGtTimeoutNs;
+#define QNT_GT_FAULT t_gt_fault
+#define QNT_GT_TIMEOUT t_gt_timeout_ns
+#else
+#define QNT_GT_FAULT 0
+#define QNT_GT_TIMEOUT kGtTimeoutNs
+#endif
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -562,26 +651,39 @@ cudaError_t gt_launch(const qnt_desc& d, const void* codes, const void* meta, lo
                       int* st, cudaStream_t s, bool* handled) {
   const int Mpad = (M + 15) / 16 * 16;
   int nst = 0;
-  for (int k = kGtMaxStages; k >= 2 && !nst; --k)
+  for (int k = kGtMaxStages / kGtGroups * kGtGroups; k >= 2 * kGtGroups && !nst; k -= kGtGroups)
     if (gt_smem(Mpad, k).total <= (size_t)kMaxDynSmem) nst = k;
   if (!nst) return cudaSuccess;
   auto enc = encode_fn();
   if (!enc) return cudaSuccess;
-  CUtensorMap map;
-  const cuuint64_t dims[2] = {(cuuint64_t)d.K, (cuuint64_t)M};
-  const cuuint64_t strides[1] = {(cuuint64_t)d.K * 2};
-  const cuuint32_t box[2] = {64u, (cuuint32_t)Mpad};
-  const cuuint32_t estr[2] = {1u, 1u};
-  const CUresult cr = enc(&map, BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-                          const_cast<void*>(X), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (cr != CUDA_SUCCESS) return cudaSuccess;   // not handled
+  // X: [M][K] fp16 / bf16, boxes of 64 columns x Mpad rows, 128-byte swizzle
+  CUtensorMap xmap, cmap;
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)d.K, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)d.K * 2};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)Mpad};
+    const cuuint32_t estr[2] = {1u, 1u};
+    if (enc(&xmap, BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(X),
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaSuccess;   // not handled
+  }
+  // codes: row groups of 4K bytes = K 32-bit words; boxes of one block (128
+  // words) x 16 row groups, no swizzle (the layout's own chunk swizzle stays)
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)d.K, (cuuint64_t)((d.N + 7) / 8)};
+    const cuuint64_t strides[1] = {(cuuint64_t)d.K * 4};
+    const cuuint32_t box[2] = {128u, 16u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    if (enc(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(codes), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaSuccess;
+  }
   auto kfn = gemm_tc_kernel<FMT, G, BF16>;
   cudaError_t e = configure_smem(reinterpret_cast<const void*>(kfn));
   if (e != cudaSuccess) return e;
   GtArgs a;
-  a.codes = static_cast<const uint8_t*>(codes);
   a.meta = static_cast<const uint8_t*>(meta);
   a.Y = Y;
   a.z0 = z0;
@@ -590,8 +692,13 @@ cudaError_t gt_launch(const qnt_desc& d, const void* codes, const void* meta, lo
   a.M = M;
   a.Mpad = Mpad;
   a.nstages = nst;
+  a.nissuers = Mpad <= 64 ? 4 : 2;   // accumulators of Mpad columns each, at most 256 columns
+  a.cola = a.nissuers * Mpad;
+  a.naslots = min(kGtMaxASlots, ((int)kGtTmemCols - a.cola) / 64) / kGtGroups * kGtGroups;
   a.xbf16 = BF16 ? 1 : 0;
   a.status = st;
+  a.timeout_ns = QNT_GT_TIMEOUT;
+  a.fault = QNT_GT_FAULT;
   *handled = true;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((d.N + kGtRows - 1) / kGtRows);
@@ -603,12 +710,12 @@ cudaError_t gt_launch(const qnt_desc& d, const void* codes, const void* meta, lo
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kfn, map, a);
+  return cudaLaunchKernelEx(&cfg, kfn, xmap, cmap, a);
 }
 
 }  // namespace
 
-// 9..128 activation rows, 4-bit formats, one pass over the weights.
+// 1..128 activation rows (dispatched for 3..128), 4-bit formats, one pass over the weights.
 cudaError_t launch_gemm_tc(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
                            int M, int xbf16, int* st, cudaStream_t s, bool* handled) {
   *handled = false;
@@ -637,5 +744,12 @@ cudaError_t launch_gemm_tc(const qnt_desc& d, const void* codes, const void* met
   }
 #undef QNT_GT
 }
+
+#ifdef QNT_TEST_FAULTS
+void set_test_gemm_fault(int fault, unsigned long long timeout_ns) {
+  t_gt_fault = fault;
+  t_gt_timeout_ns = timeout_ns;
+}
+#endif
 
 }  // namespace qnt

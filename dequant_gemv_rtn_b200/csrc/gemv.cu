@@ -8,9 +8,9 @@
 // into FP16 with bit-level operations, fused with the dot product) describe:
 //   y[m][n] = sum_k dq(code[n][k], meta[n][k/g]) * x[m][k].
 //
-// The CUDA-core multi-vector kernel: INT8 and FP16 weights, small batches of
-// FP4 / AFPQ, and batches too large for the tcgen05 kernel (gemv_tc.cu) take
-// it.  One CTA of 16 warps per SM owns a contiguous range of rows.
+// The CUDA-core multi-vector kernel: INT8 and FP16 weights at any batch and
+// the 4-bit formats at batch 2 take it.  One CTA of 16 warps per SM owns a
+// contiguous range of rows.
 //  * Activations are staged once per CTA with bulk copies; bf16 vectors are
 //    rescaled by an exact power of two into fp16 range.
 //  * A work item is (2 rows) x (2048 bytes of each row); each warp streams its

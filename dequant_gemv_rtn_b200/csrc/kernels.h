@@ -44,6 +44,8 @@ cudaError_t launch_gemv_seq_noalloc(const qnt_seq_step* steps, int n, int xbf16,
 // Test builds only (gemv1.cu): inject `fault` into this thread's next batch-1 /
 // sequence launches and use `timeout_ns` as their wait limit.
 void set_test_fault(int fault, unsigned long long timeout_ns);
+// Test builds only (gemm_tc.cu): the same for this thread's next tcgen05 GEMM launches.
+void set_test_gemm_fault(int fault, unsigned long long timeout_ns);
 #endif
 
 // An empty kernel: the next kernel in the stream cannot overlap the ones before it.
@@ -52,12 +54,6 @@ cudaError_t launch_stream_fence(cudaStream_t s);
 // Y[m] = W x[m] for 1 <= M <= 128 on the tensor cores in one pass over the
 // weights (gemm_tc.cu, 4-bit formats).  *handled = false when it does not apply.
 cudaError_t launch_gemm_tc(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
-                           int M, int xbf16, int* st, cudaStream_t s, bool* handled);
-
-// Y[m] = W x[m] for m < M on the tensor cores (gemv_tc.cu).  Returns with
-// *handled = false, launching nothing, when the tensor-core kernel does not
-// take this format / batch / shape.
-cudaError_t launch_gemv_tc(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
                            int M, int xbf16, int* st, cudaStream_t s, bool* handled);
 
 }  // namespace qnt

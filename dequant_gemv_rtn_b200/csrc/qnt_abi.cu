@@ -46,51 +46,29 @@ int check(const qnt_desc* d) {
 }
 
 // Y[m] = W x[m], m < M.  Kernel choice (measured on B200 with L2-cold weights):
-//   one vector, 4-bit formats         -> batch-1 kernel (mma.sync tensor cores)
-//   9..128 vectors, 4-bit formats     -> tcgen05 GEMM, one pass over the weights
-//   INT4, FP4, AFPQ 2..8 vectors;
-//   RaZeR 2 vectors                   -> CUDA-core multi-vector kernel
-//   RaZeR 3..8 vectors                -> tcgen05 kernel for up to 16 vectors
-//   INT8, FP16                        -> CUDA-core multi-vector kernel (passes of 8)
-// QNT_FORCE_SIMT=1 selects the CUDA-core multi-vector kernel everywhere and
-// QNT_FORCE_TC=1 the tensor-core kernel wherever it applies (used to test every
-// path on the same inputs).
+//   one vector, 4-bit formats       -> batch-1 kernel (mma.sync tensor cores)
+//   3..128 vectors, 4-bit formats   -> tcgen05 GEMM, one pass over the weights
+//   2 vectors, INT8, FP16           -> CUDA-core multi-vector kernel (passes of 8)
+// QNT_FORCE_SIMT=1 selects the CUDA-core multi-vector kernel everywhere (used to
+// test every path on the same inputs).
 cudaError_t dispatch_gemm(const qnt_desc& d, const void* codes, const void* meta, const void* X, void* Y, int M,
                           int xbf16, int* st, cudaStream_t s) {
-  static const int force = [] {
+  static const bool force_simt = [] {
     const char* a = std::getenv("QNT_FORCE_SIMT");
-    const char* b = std::getenv("QNT_FORCE_TC");
-    return (a && a[0] == '1') ? 1 : ((b && b[0] == '1') ? 2 : 0);
+    return a && a[0] == '1';
   }();
   const long z0 = zero_plane(d);
   bool handled = false;
   cudaError_t e = cudaSuccess;
-  if (force == 0 && M == 1) {
+  if (!force_simt && M == 1) {
     e = qnt::launch_gemv4_one(d, codes, meta, z0, X, Y, xbf16, st, s, &handled);
     if (handled || e != cudaSuccess) return e;
   }
-  if (force == 0 && M >= 9) {   // 4-bit formats: one pass over the weights on tcgen05
+  if (!force_simt && M >= 3) {
     e = qnt::launch_gemm_tc(d, codes, meta, z0, X, Y, M, xbf16, st, s, &handled);
     if (handled || e != cudaSuccess) return e;
   }
-  const bool tc = force == 2 || (force == 0 && ((d.fmt == QNT_INT4_ASYM && M > 8) || (d.fmt == QNT_FP4_RAZER && M > 2)));
-  int m0 = 0;   // vectors done
-  if (tc) {
-    // the tensor-core kernel takes up to 16 vectors per launch; larger batches
-    // run in passes of 16 (each pass streams the weights once)
-    while (m0 < M) {
-      const int mm = M - m0 < 16 ? M - m0 : 16;
-      handled = false;
-      e = qnt::launch_gemv_tc(d, codes, meta, z0, static_cast<const char*>(X) + (size_t)m0 * d.K * 2,
-                              static_cast<char*>(Y) + (size_t)m0 * d.N * 2, mm, xbf16, st, s, &handled);
-      if (e != cudaSuccess) return e;
-      if (!handled) break;
-      m0 += mm;
-    }
-    if (m0 == M) return cudaSuccess;
-  }
-  return qnt::launch_gemv_simt(d, codes, meta, z0, static_cast<const char*>(X) + (size_t)m0 * d.K * 2,
-                               static_cast<char*>(Y) + (size_t)m0 * d.N * 2, M - m0, xbf16, st, s);
+  return qnt::launch_gemv_simt(d, codes, meta, z0, X, Y, M, xbf16, st, s);
 }
 
 }  // namespace
@@ -258,6 +236,20 @@ extern "C" int qnt_test_gemv_seq_fault(const qnt_seq_step* steps, int nsteps, in
   qnt::set_test_fault(fault, timeout_ns);
   const int rc = qnt_gemv_seq(steps, nsteps, xdtype, d_work, d_status, stream);
   qnt::set_test_fault(0, 2000000000ull);
+  return rc;
+}
+
+// Test builds only: qnt_gemm (M >= 3, 4-bit formats: the tcgen05 GEMM) with a
+// fault injected and a short wait limit.  fault 1: in CTA 0 one decode warp
+// never reports stage 0 decoded, so the MMA issuers' wait for it gives up after
+// timeout_ns; the kernel reports QNT_ERR_TIMEOUT, lets the copies it issued
+// land, frees its tensor memory and returns.
+extern "C" int qnt_test_gemm_fault(const qnt_desc* desc, const void* d_codes, const void* d_meta, const void* d_X,
+                                   void* d_Y, int M, int xdtype, int* d_status, void* stream, int fault,
+                                   unsigned long long timeout_ns) {
+  qnt::set_test_gemm_fault(fault, timeout_ns);
+  const int rc = qnt_gemm(desc, d_codes, d_meta, d_X, d_Y, M, xdtype, d_status, stream);
+  qnt::set_test_gemm_fault(0, 2000000000ull);
   return rc;
 }
 #endif

@@ -79,6 +79,7 @@ struct GtArgs {
   int* status;
   unsigned long long timeout_ns;   // limit of every wait
   int fault;                       // test builds only: an injected fault (0: none)
+  int split;                       // CTAs per tile (a cluster), each over a share of K
 };
 
 struct GtSmem { size_t stage0, stage_bytes, xoff, total; };
@@ -106,13 +107,17 @@ __device__ __forceinline__ uint64_t gt_now() {
 // the critical path).  (A suspend-time hint on try_wait instead was measured to
 // wake the thread up to microseconds after the phase completed.)
 __device__ __forceinline__ bool gt_wait(uint64_t* bar, uint32_t parity, volatile int* abort_s, uint64_t timeout,
-                                        uint32_t max_sleep) {
+                                        uint32_t max_sleep, bool cluster_scope = false) {
   const uint32_t a = smem_addr(bar);
   uint64_t deadline = 0;
   for (uint32_t n = 0, ns = 0;; ++n) {
     uint32_t done;
-    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(done) : "r"(a), "r"(parity) : "memory");
+    if (cluster_scope)   // the phase was completed by arrivals (with release) from other CTAs of the cluster
+      asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+                   "selp.u32 %0, 1, 0, p;\n\t}" : "=r"(done) : "r"(a), "r"(parity) : "memory");
+    else
+      asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+                   : "=r"(done) : "r"(a), "r"(parity) : "memory");
     if (done) return true;
     if (max_sleep == 0 && (n & 63u) != 63u) continue;
     if (abort_s && *abort_s) return false;
@@ -199,6 +204,33 @@ __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* m
       " [%0], [%1, {%2, %3}], [%4], %5;"
       :: "r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_addr(bar)), "l"(pol)
       : "memory");
+}
+
+// Cluster helpers (split of K over the CTAs of a cluster; no multicast).
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of this CTA's shared-memory location `a` in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_map(uint32_t a, uint32_t rank) {
+  uint32_t d;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(rank));
+  return d;
+}
+__device__ __forceinline__ void cluster_arrive(uint32_t bar_cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(bar_cluster_addr) : "memory");
+}
+__device__ __forceinline__ float lds32f(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ void cluster_st_f32(uint32_t a, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(a), "f"(v) : "memory");
 }
 
 // packed bf16 arithmetic (one rounding each)
@@ -373,13 +405,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
   uint64_t* aempty = afull + kGtMaxASlots;                   // [A slots] the MMAs reading the slot are complete
   uint64_t* dfull = aempty + kGtMaxASlots;                   // all MMAs complete
   uint64_t* tmem_ready = dfull + 1;
+  uint64_t* red_ready = tmem_ready + 1;                      // split: the leader's ring is free for partial sums
+  uint64_t* red_full = red_ready + 1;                        // split, leader: every other CTA's partial sums landed
   uint32_t* tbase_p = reinterpret_cast<uint32_t*>(smem + 512);
   volatile int* abort_s = reinterpret_cast<volatile int*>(smem + 520);
   const int nst = A.nstages, nI = A.nissuers, nA = A.naslots;
   const GtSmem L = gt_smem(A.Mpad, nst);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int KB = A.K / 128, GK = A.K / G;
-  const int tile = blockIdx.x;
+  const int GK = A.K / G;
+  // split of K: the A.split CTAs of a cluster share a tile, CTA `crank` takes
+  // stages [s0, s0 + KB) of it; the leader (rank 0) sums the partial results
+  const int S = A.split;
+  const int crank = S > 1 ? (int)cluster_rank() : 0;
+  const int tile = blockIdx.x / S;
+  const int KBt = A.K / 128;
+  const int s0 = crank * KBt / S, KB = (crank + 1) * KBt / S - s0;
 
   if (tid == 0) {
     for (int i = 0; i < nst; ++i) {
@@ -392,11 +432,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
     }
     mbar_init_nofence(dfull, nI);
     mbar_init_nofence(tmem_ready, 1);
+    mbar_init_nofence(red_ready, 1);
+    mbar_init_nofence(red_full, S > 1 ? S - 1 : 1);
     mbar_init_fence();
     *abort_s = 0;
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   }
   __syncthreads();
+  if (S > 1) cluster_sync();   // every CTA's barriers are initialized before any remote arrival
   if (warp == kGtMmaWarp0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                  :: "r"(smem_addr(tbase_p)), "r"(kGtTmemCols) : "memory");
@@ -409,8 +452,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
     *abort_s = 1;
     report(A.status, QNT_ERR_TIMEOUT);
   };
-  auto wait = [&](uint64_t* bar, uint32_t parity, volatile int* ab, uint32_t max_sleep = 128) {
-    return gt_wait(bar, parity, ab, A.timeout_ns, max_sleep);
+  auto wait = [&](uint64_t* bar, uint32_t parity, volatile int* ab, uint32_t max_sleep = 128, bool cluster_scope = false) {
+    return gt_wait(bar, parity, ab, A.timeout_ns, max_sleep, cluster_scope);
   };
 
   if (warp == 0) {
@@ -421,12 +464,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
       auto stage_ptr = [&](int s) { return smem + L.stage0 + (size_t)(s % nst) * L.stage_bytes; };
       auto issue_codes = [&](int s) {
         mbar_expect_tx(full + s % nst, stage_tx);
-        tma_load_2d_hint(stage_ptr(s), &cmap, s * 128, tile * 16, full + s % nst, pol);
+        tma_load_2d_hint(stage_ptr(s), &cmap, (s0 + s) * 128, tile * 16, full + s % nst, pol);
       };
       auto issue_x = [&](int s) {
         uint8_t* st = stage_ptr(s);
-        tma_load_2d(st + L.xoff, &xmap, s * kGtStageK, 0, full + s % nst);
-        tma_load_2d(st + L.xoff + (size_t)A.Mpad * 128, &xmap, s * kGtStageK + 64, 0, full + s % nst);
+        tma_load_2d(st + L.xoff, &xmap, (s0 + s) * kGtStageK, 0, full + s % nst);
+        tma_load_2d(st + L.xoff + (size_t)A.Mpad * 128, &xmap, (s0 + s) * kGtStageK + 64, 0, full + s % nst);
       };
       // the first stages' codes do not depend on the preceding kernel; X does
       const int pre = min(nst, KB);
@@ -531,7 +574,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
     auto load_raw = [&](int s, uint32_t (&out)[kGps]) {
       if (s >= KB) return;
 #pragma unroll
-      for (int h = 0; h < kGps; ++h) out[h] = gt_meta_raw<FMT>(A.meta, A.z0, rowm * GK + (long)s * kGps + h);
+      for (int h = 0; h < kGps; ++h) out[h] = gt_meta_raw<FMT>(A.meta, A.z0, rowm * GK + (long)(s0 + s) * kGps + h);
     };
 #pragma unroll
     for (int u = 0; u < kPf; ++u) load_raw(grp + u * kGtGroups, raw[u]);
@@ -582,35 +625,73 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
       }
     }
     // epilogue: 16-column chunks of the accumulator rows, dealt out to the
-    // groups, summed over the accumulators
-    if (ok && wait(dfull, 0, abort_s)) {
-      tc_fence_after();
-      for (int cc = 16 * grp; cc < A.Mpad; cc += 16 * kGtGroups) {
-        float acc[16];
+    // groups, summed over the accumulators (and, split, over the cluster's CTAs)
+    const bool have = ok && wait(dfull, 0, abort_s);
+    if (have) tc_fence_after();
+    else if (!*abort_s) fail();
+    auto tmem_sum = [&](int cc, float (&acc)[16]) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) acc[e] = 0.0f;
-        for (int i = 0; i < nI; ++i) {
-          uint32_t d[16];
-          tmem_ld16(tbase + tlane + (uint32_t)(i * A.Mpad + cc), d);
-          tmem_wait_ld();
+      for (int e = 0; e < 16; ++e) acc[e] = 0.0f;
+      for (int i = 0; i < nI; ++i) {
+        uint32_t d[16];
+        tmem_ld16(tbase + tlane + (uint32_t)(i * A.Mpad + cc), d);
+        tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) acc[e] += __uint_as_float(d[e]);
+        for (int e = 0; e < 16; ++e) acc[e] += __uint_as_float(d[e]);
+      }
+    };
+    // partial sums of CTA k > 0 in the leader's ring: float [k - 1][column][row]
+    const uint32_t red0 = st0;
+    if (S > 1 && crank != 0) {
+      // wait until the leader's ring is free, write this CTA's partial sums
+      // there, then tell the leader (one arrival per CTA, after all decode warps)
+      const bool can = have && wait(red_ready, 0, abort_s, 512, true);
+      if (have && !can && !*abort_s) fail();
+      if (can) {
+        const uint32_t dst0 = cluster_map(red0, 0u);
+        for (int cc = 16 * grp; cc < A.Mpad; cc += 16 * kGtGroups) {
+          float acc[16];
+          tmem_sum(cc, acc);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            cluster_st_f32(dst0 + 4u * (uint32_t)((((crank - 1) * A.Mpad) + cc + e) * kGtRows + r), acc[e]);
         }
-        if (rowok) {
+      }
+      asm volatile("bar.sync 2, %0;" :: "r"(32 * 4 * kGtGroups) : "memory");   // the decode warps
+      if (dw == 0 && lane == 0) {
+        asm volatile("fence.acq_rel.cluster;" ::: "memory");
+        cluster_arrive(cluster_map(smem_addr(red_full), 0u));
+      }
+    } else if (have) {
+      if (S > 1 && dw == 0 && lane == 0)   // the ring is read: the other CTAs may write their partial sums
+        for (int k = 1; k < S; ++k) cluster_arrive(cluster_map(smem_addr(red_ready), (uint32_t)k));
+      bool red_ok = true;
+      if (S > 1) {
+        red_ok = wait(red_full, 0, abort_s, 512, true);
+        if (!red_ok && !*abort_s) fail();
+      }
+      if (red_ok) {
+        for (int cc = 16 * grp; cc < A.Mpad; cc += 16 * kGtGroups) {
+          float acc[16];
+          tmem_sum(cc, acc);
+          for (int k = 1; k < S; ++k)
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int m = cc + e;
-            if (m < A.M) {
-              const float v = acc[e] * unpw;
-              const size_t o = (size_t)m * A.N + row;
-              if (A.xbf16) reinterpret_cast<__nv_bfloat16*>(A.Y)[o] = __float2bfloat16_rn(v);
-              else reinterpret_cast<__half*>(A.Y)[o] = __float2half_rn(v);
+            for (int e = 0; e < 16; ++e)
+              acc[e] += lds32f(red0 + 4u * (uint32_t)((((k - 1) * A.Mpad) + cc + e) * kGtRows + r));
+          if (rowok) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int m = cc + e;
+              if (m < A.M) {
+                const float v = acc[e] * unpw;
+                const size_t o = (size_t)m * A.N + row;
+                if (A.xbf16) reinterpret_cast<__nv_bfloat16*>(A.Y)[o] = __float2bfloat16_rn(v);
+                else reinterpret_cast<__half*>(A.Y)[o] = __float2half_rn(v);
+              }
             }
           }
         }
       }
-    } else if (!*abort_s) {
-      fail();
     }
   }
   // teardown: every MMA issued has completed before tensor memory is freed
@@ -620,6 +701,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
     __syncwarp();
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(*tbase_p), "r"(kGtTmemCols) : "memory");
+  }
+  // split: no CTA leaves while another may still write into its shared memory
+  // or arrive on its barriers (every path above reaches this point: all waits
+  // are bounded)
+  if (S > 1) {
+    __syncthreads();
+    cluster_sync();
   }
 }
 
@@ -699,17 +787,31 @@ cudaError_t gt_launch(const qnt_desc& d, const void* codes, const void* meta, lo
   a.status = st;
   a.timeout_ns = QNT_GT_TIMEOUT;
   a.fault = QNT_GT_FAULT;
+  // Split K over a cluster of `split` CTAs per tile when the tiles alone would
+  // leave at least half of the SMs idle: a power of two up to 8, each CTA with
+  // at least 4 stages, and the partial sums of the other CTAs fitting in the
+  // leader's ring.
+  const int tiles = (d.N + kGtRows - 1) / kGtRows, KBt = d.K / kGtStageK;
+  const size_t ring = (size_t)nst * gt_smem(Mpad, nst).stage_bytes, part = (size_t)Mpad * kGtRows * 4;
+  int split = 1;
+  while (split < 8 && 2 * split * tiles <= num_sms() && KBt / (2 * split) >= 4 && (size_t)(2 * split - 1) * part <= ring)
+    split *= 2;
+  a.split = split;
   *handled = true;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((d.N + kGtRows - 1) / kGtRows);
+  cfg.gridDim = dim3(tiles * split);
   cfg.blockDim = dim3(kGtThreads);
   cfg.dynamicSmemBytes = gt_smem(Mpad, nst).total;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)split;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = split > 1 ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kfn, xmap, cmap, a);
 }
 

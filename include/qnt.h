@@ -199,7 +199,10 @@ int qnt_gemv(const qnt_desc* desc, const void* d_codes, const void* d_meta,
  * for 1 <= M <= 128 activation rows.
  *   d_X        device, [M][K] fp16 or bf16, row-major.
  *   d_Y        device, [M][N] in the same type, written.
- * Same accuracy statement as qnt_gemv.
+ * Same ordering rule (the immediately preceding kernel on the stream must not
+ * write d_codes or d_meta) and accuracy statement as qnt_gemv.  Batches of 3 to
+ * 128 rows of the 4-bit formats run on the tcgen05 tensor cores in one pass over
+ * the weights; d_status may also receive QNT_ERR_TIMEOUT there.
  */
 int qnt_gemm(const qnt_desc* desc, const void* d_codes, const void* d_meta,
              const void* d_X, void* d_Y, int M, int xdtype, int* d_status, void* stream);

@@ -56,10 +56,10 @@ def algo_bytes_int4(N, K, g=GROUP, M=1):
 
 STEP_BYTES = LAYERS * sum(algo_bytes_int4(N, K) for _, N, K in SHAPES)
 # DRAM bytes (read + write) of one launch of the sequence kernel over the whole
-# stack: an ncu capture of one decode layer (`--kernel-only layer`, 105.25 MB read
-# + 3.54 MB written, the kernel as built now) times the 32 layers, which stream
-# the same shapes.  None when the kernel has changed since the capture.
-TRAFFIC_PER_LAUNCH = 3_481_346_048
+# stack: an ncu capture of one decode layer (`--kernel-only layer`) times the 32
+# layers, which stream the same shapes.  None when the kernel has changed since
+# the capture.
+TRAFFIC_PER_LAUNCH = None
 
 
 def measured_peaks():

@@ -72,7 +72,7 @@ struct B1Step {
   int rot;       // rotation of the row-group split over the CTAs (balances remainders)
   int NG, KB, KBR, GK;   // row groups, blocks and item runs per row, groups per row
   int rows_cap;  // rows of the busiest CTA
-  int pad;
+  int reuse_x;   // 1: x is the previous step's x and cannot have changed since: keep its image
 };
 
 template <int MAXS>
@@ -490,8 +490,9 @@ gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
     if (consumer_bar_or(nct, *abort_s != 0)) break;
     // -- the activation image, straight from global memory (after the barrier:
     // ordered after thread 32's acquire of the producing step's completion)
-    for (int b = 2 * warp; b < KB; b += 2 * C)
-      build_x<FMT, G>(static_cast<const uint8_t*>(st.x), ximg_a, xs2_a, b, b + 1 < KB ? b + 1 : -1, P.xbf16, lane);
+    if (!st.reuse_x)
+      for (int b = 2 * warp; b < KB; b += 2 * C)
+        build_x<FMT, G>(static_cast<const uint8_t*>(st.x), ximg_a, xs2_a, b, b + 1 < KB ? b + 1 : -1, P.xbf16, lane);
     if (!mbar_wait_to(mfull, (uint32_t)j & 1u, P.timeout_ns, abort_s)) {
       if (!*abort_s) fail(QNT_ERR_TIMEOUT);
     }
@@ -756,6 +757,13 @@ cudaError_t b1_launch(const qnt_seq_step* steps, int n, int xbf16, unsigned* don
     b.GK = d.K / d.group;
     b.rows_cap = b1_rows_cap(d.N, grid);
     rot += (d.N + 7) / 8;   // rotate the remainder CTAs from step to step
+    // The activation image of step i - 1 serves step i when both read the same
+    // x and step i waits for no step that step i - 1 did not already wait for:
+    // x is then unchanged since it was imaged (a step that writes x must be
+    // waited for by the steps that read it).
+    const int dep = steps[i].wait > 0 ? i - steps[i].wait : -1;
+    const int dep_prev = i > 0 && steps[i - 1].wait > 0 ? i - 1 - steps[i - 1].wait : -1;
+    b.reuse_x = i > 0 && steps[i].x == steps[i - 1].x && d.K == steps[i - 1].desc.K && dep <= dep_prev ? 1 : 0;
   }
   P.nsteps = n;
   P.xbf16 = xbf16;

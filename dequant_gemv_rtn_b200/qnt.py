@@ -22,7 +22,7 @@ FORMATS = {"int4": QNT_INT4_ASYM, "fp4": QNT_FP4_E2M1, "afpq": QNT_FP4_AFPQ, "ra
            "int8": QNT_INT8_PERCHAN, "fp16": QNT_FP16}
 
 
-QNT_MAX_GEMV_K = 65536
+QNT_MAX_GEMV_K = 32768
 QNT_SEQ_MAX_STEPS = 256
 QNT_SEQ_NOALLOC_MAX_STEPS = 256
 

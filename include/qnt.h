@@ -51,9 +51,11 @@ extern "C" {
 
 #define QNT_VERSION 2
 
-/* Largest K that qnt_gemv, qnt_gemm and qnt_gemv_seq accept (the activation
- * vector is staged in shared memory); qnt_quantize accepts K up to 2^20. */
-#define QNT_MAX_GEMV_K 65536
+/* Largest K that qnt_gemv, qnt_gemm and qnt_gemv_seq accept: every GEMV
+ * kernel stages the activation vector (2K bytes) in shared memory next to its
+ * weight ring, and the CUDA-core kernel (INT8, FP16, batch 2) would not fit at
+ * K = 65536.  qnt_quantize accepts K up to 2^20. */
+#define QNT_MAX_GEMV_K 32768
 
 /* Weight formats.  h(.) = round-to-nearest-even to fp16; every quotient below
  * is one IEEE binary32 division; rint = round half to even; a scale that

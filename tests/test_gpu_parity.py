@@ -151,3 +151,19 @@ def test_gemm_rows_equal_gemv():
     for m in range(4):
         y = H.run_gemm(orc.FP4, N, K, g, pc, pm, Xb[m:m + 1], 0, use_gemv=True)
         H.assert_within_tol(y[0], yref[m], aref[m], f"row {m}")
+
+
+@pytest.mark.parametrize("fmt,M", [(orc.INT8, 1), (orc.FP16, 1), (orc.INT8, 3), (orc.INT4, 1), (orc.INT4, 2),
+                                   (orc.INT4, 16), (orc.RAZER, 2)])
+def test_largest_k_every_path(fmt, M):
+    """K = QNT_MAX_GEMV_K on every kernel a call can take (the batch-1 kernel,
+    the CUDA-core kernel at batch 1-3, the tcgen05 GEMM): the activation
+    vector fits in shared memory next to each kernel's weight ring."""
+    Q = H.q()
+    N, K, g = 72, Q.QNT_MAX_GEMV_K, 128
+    ref, pc, pm = _oracle_packed(fmt, N, K, g, seed=K + fmt + M)
+    xdt = M % 2
+    Xb = H.to_x_bits(synth.activations(M, K, seed=M + 11), xdt)
+    yref, aref = orc.gemm(ref, Xb, xdt)
+    y = H.run_gemm(fmt, N, K, g if fmt in FOUR else K, pc, pm, Xb, xdt, use_gemv=(M == 1))
+    H.assert_within_tol(y, yref, aref, f"largest K fmt={fmt} M={M}", xdt)

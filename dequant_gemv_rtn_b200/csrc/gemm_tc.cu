@@ -267,7 +267,7 @@ struct GtGroup {
   uint32_t s1, s2;     // fp16: scale pair (low / high nibble); bf16: scale high part; AFPQ: s+ / s-
   uint32_t s3;         // bf16: scale low part
   float fs, fs2;       // FP4 family with bf16: fp32 scale(s)
-  uint32_t sv;         // RaZeR: special value (fp16 bits)
+  uint32_t sv;         // RaZeR: twice the special value, as an fp16 pair
 };
 
 // Raw metadata of group f: AFPQ the (s+, s-) word; otherwise the fp16 scale in
@@ -320,7 +320,10 @@ __device__ __forceinline__ GtGroup gt_group(uint32_t raw, float pw) {
     }
     return c;
   }
-  if (FMT == QNT_FP4_RAZER) c.sv = ((extra & 2u) ? 0x4800u : 0x4500u) | ((extra & 1u) ? 0x8000u : 0u);   // +-8 or +-5
+  if (FMT == QNT_FP4_RAZER) {   // the pair (2 sv, 2 sv): +-16 or +-10
+    const uint32_t sv2 = ((extra & 2u) ? 0x4C00u : 0x4900u) | ((extra & 1u) ? 0x8000u : 0u);
+    c.sv = sv2 | (sv2 << 16);
+  }
   if (BF16) {
     c.fs = s;
   } else {
@@ -364,15 +367,14 @@ __device__ __forceinline__ void gt_decode_chunk(const uint4& cv, const GtGroup& 
     uint32_t h[4];
     cvt_e2m1x8(w[j], h[0], h[1], h[2], h[3]);
     if (FMT == QNT_FP4_RAZER) {
+      // codes 0b1000 (decoded as -0) take the group's special value, branch
+      // free: -0 + 0.5 * 2 sv = sv where the code is 0b1000, x + 0 elsewhere
       const uint32_t tt = (w[j] & 0x77777777u) + 0x77777777u;
-      const uint32_t spec = lop3<0x20>(w[j], tt, 0x88888888u);   // nibbles equal to 0b1000
-      if (spec) {
+      const uint32_t spec = lop3<0x20>(w[j], tt, 0x88888888u);   // bit 3 of every nibble equal to 0b1000
+      uint32_t ind[4];
+      cvt_e2m1x8(spec >> 3, ind[0], ind[1], ind[2], ind[3]);
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          if (spec & (0x8u << (8 * p))) h[p] = (h[p] & 0xFFFF0000u) | c.sv;
-          if (spec & (0x80u << (8 * p))) h[p] = (h[p] & 0x0000FFFFu) | (c.sv << 16);
-        }
-      }
+      for (int p = 0; p < 4; ++p) h[p] = hfma2(ind[p], c.sv, h[p]);
     }
 #pragma unroll
     for (int p = 0; p < 4; ++p) {

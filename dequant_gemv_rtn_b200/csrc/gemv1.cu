@@ -277,8 +277,8 @@ __device__ __forceinline__ uint32_t meta_sel2(const MetaRef& M, uint32_t fr) {
 
 // Decode word j of a lane's chunk and run MMA j of its block into d (and, for
 // AFPQ, the negative part into dn); MMA 0 starts the accumulators from zero.
-// bx: the lane's eight B registers; sv16: RaZeR special value (fp16 bits) of
-// this lane's chunk group.
+// bx: the lane's eight B registers; sv16: RaZeR: twice the special value of this
+// lane's chunk group, as an fp16 pair.
 template <int FMT>
 __device__ __forceinline__ void word_mma(uint32_t w, int j, const uint32_t (&bx)[8], float (&d)[4], float (&dn)[4],
                                          uint32_t sv16) {
@@ -292,16 +292,15 @@ __device__ __forceinline__ void word_mma(uint32_t w, int j, const uint32_t (&bx)
   uint32_t h[4];
   cvt_e2m1x8(w, h[0], h[1], h[2], h[3]);
   if (FMT == QNT_FP4_RAZER) {
-    // codes 0b1000 (decoded as -0) take the group's special value
+    // codes 0b1000 decode to -0 and take the group's special value sv, branch
+    // free: nibbles 0b0001 exactly where the code is 0b1000 convert to 0.5, and
+    // -0 + 0.5 * 2sv = sv, x + 0 * 2sv = x (sv16: the pair 2sv, 2sv)
     const uint32_t tt = (w & 0x77777777u) + 0x77777777u;
-    const uint32_t spec = lop3<0x20>(w, tt, 0x88888888u);
-    if (spec) {
+    const uint32_t spec = lop3<0x20>(w, tt, 0x88888888u);   // bit 3 of every nibble equal to 0b1000
+    uint32_t ind[4];
+    cvt_e2m1x8(spec >> 3, ind[0], ind[1], ind[2], ind[3]);
 #pragma unroll
-      for (int pp = 0; pp < 4; ++pp) {
-        if (spec & (0x8u << (8 * pp))) h[pp] = (h[pp] & 0xFFFF0000u) | sv16;
-        if (spec & (0x80u << (8 * pp))) h[pp] = (h[pp] & 0x0000FFFFu) | (sv16 << 16);
-      }
-    }
+    for (int pp = 0; pp < 4; ++pp) h[pp] = hfma2(ind[pp], sv16, h[pp]);
   }
   if (FMT == QNT_FP4_AFPQ) {
     uint32_t hp[4], hn[4];
@@ -560,7 +559,8 @@ gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
             sv16[i] = 0u;
             if (FMT == QNT_FP4_RAZER) {
               const uint32_t sel = meta_sel2(M, fr0 - eh + (uint32_t)(q + NQ * i) + rz);
-              sv16[i] = ((sel & 2u) ? 0x4800u : 0x4500u) | ((sel & 1u) ? 0x8000u : 0u);
+              const uint32_t sv2 = ((sel & 2u) ? 0x4C00u : 0x4900u) | ((sel & 1u) ? 0x8000u : 0u);   // 2 sv: +-16 or +-10
+              sv16[i] = sv2 | (sv2 << 16);
             }
           }
           float d[S][4], dn[S][4];
@@ -620,7 +620,8 @@ gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
               uint32_t sv = 0u;
               if (FMT == QNT_FP4_RAZER) {
                 const uint32_t sel = meta_sel2(M, fr0 - eh + (uint32_t)(blk * GPB) + rz);
-                sv = ((sel & 2u) ? 0x4800u : 0x4500u) | ((sel & 1u) ? 0x8000u : 0u);   // +-8 or +-5
+                const uint32_t sv2 = ((sel & 2u) ? 0x4C00u : 0x4900u) | ((sel & 1u) ? 0x8000u : 0u);   // 2 sv: +-16 or +-10
+                sv = sv2 | (sv2 << 16);
               }
 #pragma unroll
               for (int jj = 0; jj < 4; ++jj) word_mma<FMT>((&cv.x)[jj], jj, bx, d[i], dn[i], sv);

@@ -587,12 +587,41 @@ def run_extra_configs(args):
         Xs = {K: synth.activations_device(M, K, seed=K, dtype=torch.float16) for K in (4096, 11008)}
         Ys = {N: torch.empty((M, N), dtype=torch.float16, device="cuda") for N in (4096, 11008, 32000)}
 
-        def run_stack(s, M=M, Xs=Xs, Ys=Ys):
-            for fmt, N, K, d, c, m in stack:
-                if M == 1:
-                    Q.qnt_gemv(d, c, m, Xs[K], Ys[N], 0, st, s)
+        # batch 1: each run of INT4 modules is one qnt_gemv_seq call with the data
+        # dependencies of a decode layer (q, k, v read the previous layer's down
+        # output; o reads attention over q, k, v; gate and up read o's; down reads
+        # gate's and up's), the INT8 modules qnt_gemv calls between them (each
+        # module its own y, as the sequence call requires)
+        producer = {0: -1, 1: -1, 2: -1, 3: 2, 4: 3, 5: 3, 6: 5}   # module in the layer -> producing module
+        segments = []
+        if M == 1:
+            for i, (fmt, N, K, d, c, m) in enumerate(stack):
+                y = torch.empty(N, dtype=torch.float16, device="cuda")
+                l, j = divmod(i, 7)
+                p = 7 * l + producer[j] if producer[j] >= 0 else 7 * l - 1   # global index of the producer
+                if fmt == Q.QNT_INT4_ASYM and segments and segments[-1][0] == "seq" and \
+                        len(segments[-1][1]) < Q.QNT_SEQ_MAX_STEPS:
+                    start = segments[-1][2]
+                    local = len(segments[-1][1])
+                    segments[-1][1].append((d, c, m, Xs[K], y, local - (p - start) if p >= start else 0))
+                elif fmt == Q.QNT_INT4_ASYM:
+                    segments.append(("seq", [(d, c, m, Xs[K], y, 0)], i))
                 else:
-                    Q.qnt_gemm(d, c, m, Xs[K], Ys[N], M, 0, st, s)
+                    segments.append(("one", (d, c, m, Xs[K], y), i))
+            segments = [(kind, (Q.seq_steps(v), torch.zeros(Q.qnt_gemv_seq_work_bytes(len(v)), dtype=torch.uint8,
+                                                             device="cuda")) if kind == "seq" else v)
+                        for kind, v, _ in segments]
+
+        def run_stack(s, M=M, Xs=Xs, Ys=Ys, segments=segments):
+            if M == 1:
+                for kind, v in segments:
+                    if kind == "seq":
+                        Q.qnt_gemv_seq(v[0], 0, v[1], st, s)
+                    else:
+                        Q.qnt_gemv(*v, 0, st, s)
+                return
+            for fmt, N, K, d, c, m in stack:
+                Q.qnt_gemm(d, c, m, Xs[K], Ys[N], M, 0, st, s)
 
         def run_head(s, M=M, Xs=Xs, Ys=Ys):
             d, c, m = head
@@ -607,8 +636,10 @@ def run_extra_configs(args):
             "p10_p90_ms": [round(pct(ms, 10), 4), round(pct(ms, 90), 4)],
             "GBps": round(stack_bytes[M] / (med * 1e-3) / 1e9, 1),
             "frac_hbm": round(stack_bytes[M] / (med * 1e-3) / 1e9 / hbm, 4),
-            "how": "224 modules (INT4 g128; INT8 per-channel down_proj in layers 0,1,30,31) as qnt_gemv / "
-                   "qnt_gemm launches in one CUDA graph"}
+            "how": ("224 modules (INT4 g128; INT8 per-channel down_proj in layers 0,1,30,31) in one CUDA graph: "
+                    + (f"{sum(k == 'seq' for k, _ in segments)} qnt_gemv_seq calls with the decode-layer "
+                       "dependencies for the INT4 runs, qnt_gemv for the INT8 modules" if M == 1 else
+                       "224 qnt_gemm launches"))}
         hm = _time_graph(torch, stream, run_head, 3, 20)
         hmed = statistics.median(hm)
         hb = algo_bytes(6, 32000, 4096, M)

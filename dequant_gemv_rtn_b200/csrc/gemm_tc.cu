@@ -402,10 +402,11 @@ __global__ void __launch_bounds__(kGtThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap cmap, const GtArgs A) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);       // [nst] codes + X landed
-  uint64_t* empty = full + kGtMaxStages;                     // [nst] the stage's MMAs are complete
+  // [nst] the stage's MMAs are complete: frees its shared-memory slot and (for
+  // stage s + nA) its A slot; one commit per issuer and stage
+  uint64_t* empty = full + kGtMaxStages;
   uint64_t* afull = empty + kGtMaxStages;                    // [A slots] A written to tensor memory
-  uint64_t* aempty = afull + kGtMaxASlots;                   // [A slots] the MMAs reading the slot are complete
-  uint64_t* dfull = aempty + kGtMaxASlots;                   // all MMAs complete
+  uint64_t* dfull = afull + kGtMaxASlots;                    // all MMAs complete
   uint64_t* tmem_ready = dfull + 1;
   uint64_t* red_ready = tmem_ready + 1;                      // split: the leader's ring is free for partial sums
   uint64_t* red_full = red_ready + 1;                        // split, leader: every other CTA's partial sums landed
@@ -428,10 +429,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
       mbar_init_nofence(full + i, 1);
       mbar_init_nofence(empty + i, nI);
     }
-    for (int i = 0; i < nA; ++i) {
-      mbar_init_nofence(afull + i, 4);
-      mbar_init_nofence(aempty + i, nI);
-    }
+    for (int i = 0; i < nA; ++i) mbar_init_nofence(afull + i, 4);
     mbar_init_nofence(dfull, nI);
     mbar_init_nofence(tmem_ready, 1);
     mbar_init_nofence(red_ready, 1);
@@ -522,7 +520,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
             tc_mma_tmem_a(dcol, acol + 8u * (uint32_t)kk, sw128_desc(b_addr), idesc, (s > 0 || kk > kk0) ? 1u : 0u);
           }
           tc_commit(empty + slot);
-          tc_commit(aempty + as);
         }
       }
       tc_commit(dfull);   // arrives once every MMA this thread issued has completed
@@ -582,7 +579,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
     for (int u = 0; u < kPf; ++u) load_raw(grp + u * kGtGroups, raw[u]);
     // ring positions of this group's next stage; nst and nA are multiples of
     // kGtGroups, so the stage that last used a slot was this group's own
-    GtRing fr, ar;
+    GtRing fr, ar, er;   // er: the stage s - nA whose completion frees stage s's A slot
+    bool er_set = false;
     fr.adv(grp, nst);
     ar.adv(grp, nA);
     for (int s0 = grp; s0 < KB && ok; s0 += kGtGroups * kPf) {
@@ -595,13 +593,20 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         for (int h = 0; h < kGps; ++h) c[h] = gt_group<FMT, BF16>(raw[u][h], pw);
         load_raw(s + kGtGroups * kPf, raw[u]);
         const int slot = fr.slot, as = ar.slot;
-        if ((s >= nA && !wait(aempty + as, ar.phase ^ 1u, abort_s)) || !wait(full + slot, fr.phase, abort_s)) {
+        // the A slot is free once stage s - nA's MMAs are complete
+        if (s >= nA && !er_set) {
+          er.slot = (s - nA) % nst;
+          er.phase = (uint32_t)((s - nA) / nst) & 1u;
+          er_set = true;
+        }
+        if ((s >= nA && !wait(empty + er.slot, er.phase, abort_s)) || !wait(full + slot, fr.phase, abort_s)) {
           if (!*abort_s) fail();
           ok = false;
           break;
         }
         fr.adv(kGtGroups, nst);
         ar.adv(kGtGroups, nA);
+        if (er_set) er.adv(kGtGroups, nst);
         tc_fence_after();
         const uint32_t cbase = st0 + (uint32_t)(slot * L.stage_bytes) + (uint32_t)(rg * 512 + 64 * i8);
         const uint32_t abase = tbase + tlane + (uint32_t)A.cola + 64u * (uint32_t)as;
@@ -782,7 +787,13 @@ cudaError_t gt_launch(const qnt_desc& d, const void* codes, const void* meta, lo
   a.M = M;
   a.Mpad = Mpad;
   a.nstages = nst;
-  a.nissuers = Mpad <= 64 ? 4 : 2;   // accumulators of Mpad columns each, at most 256 columns
+#ifndef QNT_GT_ISSUERS
+#define QNT_GT_ISSUERS 4
+#endif
+  // MMA issuers (one accumulator of Mpad columns each): a small-N MMA keeps its
+  // issuing thread ~60 cycles, so four threads share each stage's eight MMAs
+  // (measured on 8192 x 28672, M = 16: one issuer 104 us, two 82, four 72)
+  a.nissuers = min(QNT_GT_ISSUERS, Mpad <= 64 ? 4 : 2);
   a.cola = a.nissuers * Mpad;
   a.naslots = min(kGtMaxASlots, ((int)kGtTmemCols - a.cola) / 64) / kGtGroups * kGtGroups;
   a.xbf16 = BF16 ? 1 : 0;

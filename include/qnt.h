@@ -49,7 +49,7 @@
 extern "C" {
 #endif
 
-#define QNT_VERSION 2
+#define QNT_VERSION 3
 
 /* Largest K that qnt_gemv, qnt_gemm and qnt_gemv_seq accept: every GEMV
  * kernel stages the activation vector (2K bytes) in shared memory next to its

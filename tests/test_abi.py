@@ -40,7 +40,7 @@ def test_exports_every_declared_symbol(q):
 
 
 def test_version_and_strerror(q):
-    assert q.qnt_version() == 2
+    assert q.qnt_version() == 3
     for c in range(8):
         assert q.qnt_strerror(c)
     assert "unknown" in q.qnt_strerror(99)

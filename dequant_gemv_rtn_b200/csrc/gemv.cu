@@ -329,7 +329,6 @@ gemv_simt_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ 
       }
       continue;
     }
-    const long ra = r_lo + 2 * un;
     const int nch = (int)(min((long)kRangeBytes, rowbytes - (long)kr * kRangeBytes) / 16);   // chunks in range
     float acc[2][MB][2];
 #pragma unroll

@@ -553,14 +553,14 @@ def run_extra_configs(args):
     for fmt, fname in ((2, "fp4"), (3, "afpq"), (4, "razer")):
         N, K = 14336, 4096
         copies = [_quantized(Q, torch, synth, fmt, N, K, GROUP, 40 + i, st) for i in range(ncopies(algo_bytes(fmt, N, K, 1)))]
-        for M in (1, 4):
+        for M in (1, 2, 4):
             out[f"{fname}_g128_{K}x{N}_b{M}"] = timed(fname, fmt, N, K, M, 0, copies)
         del copies
         torch.cuda.empty_cache()
     # Llama-70B INT4 g128, bf16 activations, M sweep
     for N, K in ((10240, 8192), (28672, 8192), (8192, 28672)):
         copies = [_quantized(Q, torch, synth, 1, N, K, GROUP, 60 + i, st) for i in range(ncopies(algo_bytes(1, N, K, 1)))]
-        for M in (1, 8, 16, 32, 64, 128):
+        for M in (1, 2, 4, 8, 16, 32, 64, 128):
             out[f"int4_g128_{K}x{N}_bf16_M{M}"] = timed("llama70b", 1, N, K, M, 1, copies)
         del copies
         torch.cuda.empty_cache()

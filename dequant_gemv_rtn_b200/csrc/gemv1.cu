@@ -88,19 +88,22 @@ struct B1Params {
   unsigned* done;   // [nsteps] completion counters, then one abort word (sequence only)
   int* status;
   unsigned long long timeout_ns;
+  int nvec;         // activation vectors of a several-vector launch (MV > 1), else 1
 };
 
 // The weight rings, the activation image with its table of per-(block, group)
 // factors, the per-row partial sums and the staged metadata window.
+// With mv activation vectors (several-vector launches) the image, the factor
+// table and the partial sums are held once per vector, one after another.
 struct B1Smem { size_t ring, ximg, xs2, part, meta, total; };
 constexpr int kB1SlotBytes = kB1Blocks * 512;
-__host__ __device__ inline B1Smem b1_smem(int depth, int kmax, int gpb, int part_cap, int meta_cap) {
+__host__ __device__ inline B1Smem b1_smem(int depth, int kmax, int gpb, int part_cap, int meta_cap, int mv = 1) {
   B1Smem L;
   L.ring = kB1Ctrl;
   L.ximg = L.ring + (size_t)kB1Warps * depth * kB1SlotBytes;
-  L.xs2 = align16(L.ximg + (size_t)kmax * 2);
-  L.part = align16(L.xs2 + (size_t)(kmax / 128) * gpb * 8);
-  L.meta = align16(L.part + (size_t)part_cap * 4);
+  L.xs2 = align16(L.ximg + (size_t)mv * kmax * 2);
+  L.part = align16(L.xs2 + (size_t)mv * (kmax / 128) * gpb * 8);
+  L.meta = align16(L.part + (size_t)mv * part_cap * 4);
   L.total = align16(L.meta + (size_t)meta_cap);
   return L;
 }
@@ -202,14 +205,15 @@ __device__ __forceinline__ uint32_t xf_off(int b, int r, int s, int j, int hf) {
 // over the group), c = 2^24 for INT4 (undoes the subnormal encoding), else 1.
 template <int FMT, int G>
 __device__ __forceinline__ void build_x(const uint8_t* xg, uint32_t ximg, uint32_t xs2, int b0, int b1, int xbf16,
-                                        int lane) {
+                                        int lane, bool zero = false) {
   constexpr int GPB = 128 / G;
   const int bb[2] = {b0, b1 >= 0 ? b1 : b0};
   float v[2][4], sg[2];
   uint32_t am[2];
   uint2 raws[2];
 #pragma unroll
-  for (int q = 0; q < 2; ++q) raws[q] = ldg_cg64(xg + 256 * bb[q] + 8 * lane);   // L2: x may be another CTA's y
+  for (int q = 0; q < 2; ++q)   // L2: x may be another CTA's y; zero: an image of zeros (no vector)
+    raws[q] = zero ? make_uint2(0u, 0u) : ldg_cg64(xg + 256 * bb[q] + 8 * lane);
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
     const uint2 raw = raws[q];
@@ -324,11 +328,11 @@ __device__ __forceinline__ void word_mma(uint32_t w, int j, const uint32_t (&bx)
 }
 
 // ------------------------------------------------------------------ kernel
-template <int FMT, int G, int MAXS>
+template <int FMT, int G, int MAXS, int MV>
 __global__ void __launch_bounds__(kB1Threads, 1)
 gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
   constexpr int GPB = 128 / G;        // groups per block
-  constexpr int S = 4 / GPB;          // blocks per set (accumulators)
+  constexpr int S = 4 / (GPB * MV);   // blocks per set (accumulators)
   constexpr int NQ = kB1Blocks / S;   // sets per full item
   constexpr int RB = kB1Blocks;
   constexpr int C = kB1Warps;
@@ -338,7 +342,7 @@ gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
   uint64_t* mfull = full + C * kB1MaxDepth;                // staged metadata landed
   volatile int* abort_s = reinterpret_cast<volatile int*>(smem + 1280);
   const int D = P.depth;
-  const B1Smem L = b1_smem(D, P.kmax, GPB, P.part_cap, P.meta_cap);
+  const B1Smem L = b1_smem(D, P.kmax, GPB, P.part_cap, P.meta_cap, MV);
   const uint32_t sbase = smem_addr(smem);
   const uint32_t ximg_a = sbase + (uint32_t)L.ximg, xs2_a = sbase + (uint32_t)L.xs2;
   float* part = reinterpret_cast<float*>(smem + L.part);
@@ -452,8 +456,12 @@ gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
   const int g = lane >> 2, r = lane & 3;
   const int hp = lane >> 3;                                    // B column pair of this lane
   const bool bload = (r * GPB) / 4 == hp % GPB;                // this lane's chunk lies in the pair's group
-  const int bsel = hp / GPB;                                   // block of the set that feeds the pair
-  const int ei = r / GPB, eh = r % GPB;                        // epilogue: accumulator, group in block
+  const int bsel = hp / (GPB * MV);                            // block of the set that feeds the pair
+  const int ei = r / (GPB * MV), eh = r % GPB;                 // epilogue: accumulator, group in block
+  // several vectors (MV > 1, g = 128): column pair hp carries vector hp % MV of
+  // block hp / MV of the set, and lane 4g + r's result belongs to vector r % MV
+  const int vb = hp % MV, ve = r % MV;
+  const int IMGV = 2 * P.kmax, XSV = (P.kmax / 128) * GPB * 8;   // bytes per vector: image, factor table
   const uint32_t coff = 64u * g + 16u * (uint32_t)(r ^ ((g >> 1) & 3));
   const uint32_t xoff = 16u * (uint32_t)(4 * ((lane >> 2) & 1) + r);
   const uint32_t rz = (uint32_t)((r * GPB) / 4);              // group of this lane's chunk within a block
@@ -489,9 +497,17 @@ gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
     if (consumer_bar_or(nct, *abort_s != 0)) break;
     // -- the activation image, straight from global memory (after the barrier:
     // ordered after thread 32's acquire of the producing step's completion)
-    if (!st.reuse_x)
-      for (int b = 2 * warp; b < KB; b += 2 * C)
-        build_x<FMT, G>(static_cast<const uint8_t*>(st.x), ximg_a, xs2_a, b, b + 1 < KB ? b + 1 : -1, P.xbf16, lane);
+    if (!st.reuse_x) {
+      if constexpr (MV == 1) {
+        for (int b = 2 * warp; b < KB; b += 2 * C)
+          build_x<FMT, G>(static_cast<const uint8_t*>(st.x), ximg_a, xs2_a, b, b + 1 < KB ? b + 1 : -1, P.xbf16, lane);
+      } else {   // vector v of x is row v of [M][K]; vectors past M get an image of zeros
+        for (int v = 0; v < MV; ++v)
+          for (int b = 2 * warp; b < KB; b += 2 * C)
+            build_x<FMT, G>(static_cast<const uint8_t*>(st.x) + (size_t)v * 2 * st.K, ximg_a + (uint32_t)(v * IMGV),
+                            xs2_a + (uint32_t)(v * XSV), b, b + 1 < KB ? b + 1 : -1, P.xbf16, lane, v >= P.nvec);
+      }
+    }
     if (!mbar_wait_to(mfull, (uint32_t)j & 1u, P.timeout_ns, abort_s)) {
       if (!*abort_s) fail(QNT_ERR_TIMEOUT);
     }
@@ -525,7 +541,8 @@ gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
       }
       const uint32_t ca = sbase + (uint32_t)L.ring + (uint32_t)slot * (uint32_t)kB1SlotBytes + coff;
       float yacc = 0.0f;
-      if (nb == RB && G == 128 && FMT != QNT_FP4_AFPQ && (GK & 1) == 0) {
+      if (MV > 1 || (nb == RB && G == 128 && FMT != QNT_FP4_AFPQ && (GK & 1) == 0)) {
+       if constexpr (MV == 1) {
         // ---- full item, g = 128, an even number of groups per row: the lane's
         // epilogue blocks are ei * NQ + q, q < NQ (two consecutive groups of its
         // row, the first of even index, so both scales are one aligned 32-bit
@@ -574,8 +591,61 @@ gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
             if (ei == i) v = d[i][0] + d[i][3];
           yacc += ea[q] * v - eb[q];
         }
+       } else {
+        // ---- several vectors (g = 128, full items, not AFPQ: the launcher's
+        // conditions).  Set q holds blocks q + NQ i (i < S); the lane's epilogue
+        // blocks are NQ ei + q, q < NQ: NQ consecutive groups of its row whose
+        // scales (and INT4 zero points) are one aligned load, as the group index
+        // of the first is a multiple of NQ (K is a multiple of 1024).
+        static_assert(G == 128 && FMT != QNT_FP4_AFPQ, "several vectors: g = 128, not AFPQ");
+        const uint32_t fe = fr0 + (uint32_t)(NQ * ei);
+        uint32_t sw[NQ / 2];                                   // the NQ fp16 scales, two per word
+        if constexpr (NQ == 8) {
+          const uint4 t = lds128a(M.ms_a + 2u * fe);
+          sw[0] = t.x; sw[1] = t.y; sw[2] = t.z; sw[3] = t.w;
+        } else {
+          const uint2 t = lds64a(M.ms_a + 2u * fe);
+          sw[0] = t.x; sw[1] = t.y;
+        }
+        uint32_t zw = 0u;                                      // INT4: the NQ zero points, a nibble each
+        if (FMT == QNT_INT4_ASYM) zw = NQ == 8 ? lds32a(M.mz_a + (fe >> 1)) : lds16a(M.mz_a + (fe >> 1));
+        const uint32_t xsv = xs2_a + (uint32_t)(ve * XSV) + 8u * (uint32_t)(b0 + NQ * ei);   // vector ve's factors
+        const uint32_t xa = ximg_a + (uint32_t)(vb * IMGV) + 256u * (uint32_t)(b0 + NQ * bsel) + xoff;
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          uint4 cv[S];
+#pragma unroll
+          for (int i = 0; i < S; ++i) cv[i] = lds128a(ca + 512u * (uint32_t)(q + NQ * i));
+          const uint4 x0 = lds128a(xa + 256u * q), x1 = lds128a(xa + 256u * q + 128u);
+          const uint32_t bx[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+          uint32_t sv16[S];
+#pragma unroll
+          for (int i = 0; i < S; ++i) {
+            sv16[i] = 0u;
+            if (FMT == QNT_FP4_RAZER) {
+              const uint32_t sel = meta_sel2(M, fr0 + (uint32_t)(q + NQ * i));
+              const uint32_t sv2 = ((sel & 2u) ? 0x4C00u : 0x4900u) | ((sel & 1u) ? 0x8000u : 0u);   // 2 sv: +-16 or +-10
+              sv16[i] = sv2 | (sv2 << 16);
+            }
+          }
+          float d[S][4], dn[S][4];
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+            for (int i = 0; i < S; ++i) word_mma<FMT>((&cv[i].x)[jj], jj, bx, d[i], dn[i], sv16[i]);
+          float v = d[0][0] + d[0][3];
+#pragma unroll
+          for (int i = 1; i < S; ++i)
+            if (ei == i) v = d[i][0] + d[i][3];
+          const float2 sc = lds64fa(xsv + 8u * q);             // (c / 2^e, group sum of x) of vector ve
+          const float sq = h2f((sw[q >> 1] >> (16 * (q & 1))) & 0xFFFFu);
+          const float zq = FMT == QNT_INT4_ASYM ? (float)((zw >> (4 * q)) & 15u) : 0.0f;
+          yacc += sq * (sc.x * v - zq * sc.y);
+        }
         if (!rowok) yacc = 0.0f;
+       }
       } else {
+       if constexpr (MV == 1) {
         // ---- general item (g < 128, AFPQ, or the last run of K of a row)
         auto set_epilogue = [&](int q, const float (&d)[S][4], const float (&dn)[S][4]) {
           // accumulator ei holds this lane's (row g, block q + NQ ei, group eh)
@@ -629,6 +699,7 @@ gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
           }
           set_epilogue(q, d, dn);
         }
+       }
       }
       // the slot is read: refill it with this warp's item D ahead
       __syncwarp();
@@ -638,9 +709,14 @@ gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
         fence_proxy_async();
         issue_next();
       }
-      yacc += __shfl_xor_sync(0xffffffffu, yacc, 1);
-      yacc += __shfl_xor_sync(0xffffffffu, yacc, 2);
-      if (r == 0 && rowok) part[rl * KBR + br] = yacc;
+      if constexpr (MV == 1) {
+        yacc += __shfl_xor_sync(0xffffffffu, yacc, 1);
+        yacc += __shfl_xor_sync(0xffffffffu, yacc, 2);
+        if (r == 0 && rowok) part[rl * KBR + br] = yacc;
+      } else {   // lanes r and r ^ 2 hold the same vector when MV = 2; lane r < MV ends with vector r
+        if (MV == 2) yacc += __shfl_xor_sync(0xffffffffu, yacc, 2);
+        if (r < MV && rowok) part[r * P.part_cap + rl * KBR + br] = yacc;
+      }
       u += du;
       br += dbr;
       if (br >= KBR) { br -= KBR; ++u; }
@@ -650,11 +726,22 @@ gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
     // which lands while the step's completion propagates
     if (tid == 32 && j + 1 < P.nsteps) issue_meta(j + 1);
     // -- this CTA's rows of y, the partial sums combined in a fixed order
-    for (int rr = tid; rr < nrows; rr += nct) {
-      float v = 0.0f;
-      for (int b = 0; b < KBR; ++b) v += part[rr * KBR + b];
-      if (P.xbf16) reinterpret_cast<__nv_bfloat16*>(st.y)[r_lo + rr] = __float2bfloat16_rn(v);
-      else reinterpret_cast<__half*>(st.y)[r_lo + rr] = __float2half_rn(v);
+    if constexpr (MV == 1) {
+      for (int rr = tid; rr < nrows; rr += nct) {
+        float v = 0.0f;
+        for (int b = 0; b < KBR; ++b) v += part[rr * KBR + b];
+        if (P.xbf16) reinterpret_cast<__nv_bfloat16*>(st.y)[r_lo + rr] = __float2bfloat16_rn(v);
+        else reinterpret_cast<__half*>(st.y)[r_lo + rr] = __float2half_rn(v);
+      }
+    } else {   // vector v's outputs are row v of [M][N]
+      for (int rr = tid; rr < nrows; rr += nct)
+        for (int vv = 0; vv < P.nvec; ++vv) {
+          float v = 0.0f;
+          for (int b = 0; b < KBR; ++b) v += part[vv * P.part_cap + rr * KBR + b];
+          const long o = (long)vv * st.N + r_lo + rr;
+          if (P.xbf16) reinterpret_cast<__nv_bfloat16*>(st.y)[o] = __float2bfloat16_rn(v);
+          else reinterpret_cast<__half*>(st.y)[o] = __float2half_rn(v);
+        }
     }
     consumer_bar(nct);
 #ifdef QNT_TEST_FAULTS
@@ -697,7 +784,7 @@ namespace {
 // Shared-memory plan of a launch: the deepest per-warp ring that fits with the
 // activation image and two staged metadata windows.  depth = 0 if it does not fit.
 struct B1Plan { int depth, kmax, meta_cap, part_cap; size_t smem; };
-template <int FMT, int G>
+template <int FMT, int G, int MV>
 B1Plan b1_plan(const qnt_seq_step* steps, int n, int grid) {
   B1Plan p = {0, 0, 0, 0, 0};
   size_t meta = 0;
@@ -713,7 +800,7 @@ B1Plan b1_plan(const qnt_seq_step* steps, int n, int grid) {
   p.meta_cap = (int)align16(meta);
   constexpr int GPB = 128 / G;
   for (int dp = kB1MaxDepth; dp >= 1; --dp) {
-    const size_t tot = b1_smem(dp, p.kmax, GPB, p.part_cap, p.meta_cap).total;
+    const size_t tot = b1_smem(dp, p.kmax, GPB, p.part_cap, p.meta_cap, MV).total;
     if (tot <= (size_t)kMaxDynSmem) {
       p.depth = dp;
       p.smem = tot;
@@ -723,9 +810,12 @@ B1Plan b1_plan(const qnt_seq_step* steps, int n, int grid) {
   return p;
 }
 
-template <int FMT, int G, int MAXS>
+// MV > 1: one step whose x is [nvec][K] and y [nvec][N] (nvec <= MV).  A plan
+// with a single ring slot per warp is still taken: measured on B200 it beats the
+// other kernels (M = 4 on K = 8192, N = 28672: 33 us against 71 on tcgen05).
+template <int FMT, int G, int MAXS, int MV = 1>
 cudaError_t b1_launch(const qnt_seq_step* steps, int n, int xbf16, unsigned* done, int* st, cudaStream_t s,
-                      bool cooperative, bool* handled) {
+                      bool cooperative, bool* handled, int nvec = 1) {
   const int sms = num_sms();
   long maxng = 1;
   for (int i = 0; i < n; ++i) maxng = maxng > (steps[i].desc.N + 7) / 8 ? maxng : (steps[i].desc.N + 7) / 8;
@@ -733,9 +823,9 @@ cudaError_t b1_launch(const qnt_seq_step* steps, int n, int xbf16, unsigned* don
   static B1Params<MAXS> P;   // large: built in static storage, copied by the launch
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);
-  const B1Plan p = b1_plan<FMT, G>(steps, n, grid);
-  if (!p.depth) return cudaSuccess;   // not handled: the activation vector and metadata do not fit
-  auto kfn = gemv1_kernel<FMT, G, MAXS>;
+  const B1Plan p = b1_plan<FMT, G, MV>(steps, n, grid);
+  if (!p.depth) return cudaSuccess;   // not handled: the activations and metadata do not fit
+  auto kfn = gemv1_kernel<FMT, G, MAXS, MV>;
   cudaError_t e = configure_smem(reinterpret_cast<const void*>(kfn));
   if (e != cudaSuccess) return e;
   std::memset(&P, 0, sizeof(P));
@@ -776,6 +866,7 @@ cudaError_t b1_launch(const qnt_seq_step* steps, int n, int xbf16, unsigned* don
   P.status = st;
   P.fault = QNT_B1_FAULT;
   P.timeout_ns = QNT_B1_TIMEOUT;
+  P.nvec = nvec;
   *handled = true;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -827,6 +918,29 @@ cudaError_t launch_gemv4_one(const qnt_desc& d, const void* codes, const void* m
   one.y = Y;
   one.wait = 0;
   return b1_dispatch<1>(&one, 1, xbf16, nullptr, st, s, false, handled);
+}
+
+cudaError_t launch_gemv1_multi(const qnt_desc& d, const void* codes, const void* meta, const void* X, void* Y, int M,
+                              int xbf16, int* st, cudaStream_t s, bool* handled) {
+  *handled = false;
+  if (M < 2 || M > 4 || d.group != 128 || d.K % 1024 != 0) return cudaSuccess;
+  qnt_seq_step one = {};
+  one.desc = d;
+  one.codes = codes;
+  one.meta = meta;
+  one.x = X;
+  one.y = Y;
+  one.wait = 0;
+#define QNT_B1M(FMT)                                                                                       \
+  return M == 2 ? b1_launch<FMT, 128, 1, 2>(&one, 1, xbf16, nullptr, st, s, false, handled, M)            \
+                : b1_launch<FMT, 128, 1, 4>(&one, 1, xbf16, nullptr, st, s, false, handled, M);
+  switch (d.fmt) {
+    case QNT_INT4_ASYM: QNT_B1M(QNT_INT4_ASYM)
+    case QNT_FP4_E2M1: QNT_B1M(QNT_FP4_E2M1)
+    case QNT_FP4_RAZER: QNT_B1M(QNT_FP4_RAZER)
+    default: return cudaSuccess;   // AFPQ: not handled here
+  }
+#undef QNT_B1M
 }
 
 cudaError_t launch_gemv_seq(const qnt_seq_step* steps, int n, int xbf16, void* work, int* st, cudaStream_t s,

@@ -47,8 +47,10 @@ int check(const qnt_desc* d) {
 
 // Y[m] = W x[m], m < M.  Kernel choice (measured on B200 with L2-cold weights):
 //   one vector, 4-bit formats       -> batch-1 kernel (mma.sync tensor cores)
+//   2..4 vectors, INT4 / FP4 / RaZeR, group 128, K a multiple of 1024
+//                                   -> the batch-1 kernel, the vectors sharing its MMAs
 //   3..128 vectors, 4-bit formats   -> tcgen05 GEMM, one pass over the weights
-//   2 vectors, INT8, FP16           -> CUDA-core multi-vector kernel (passes of 8)
+//   2 vectors otherwise, INT8, FP16 -> CUDA-core multi-vector kernel (passes of 8)
 // QNT_FORCE_SIMT=1 selects the CUDA-core multi-vector kernel everywhere (used to
 // test every path on the same inputs).
 cudaError_t dispatch_gemm(const qnt_desc& d, const void* codes, const void* meta, const void* X, void* Y, int M,
@@ -62,6 +64,10 @@ cudaError_t dispatch_gemm(const qnt_desc& d, const void* codes, const void* meta
   cudaError_t e = cudaSuccess;
   if (!force_simt && M == 1) {
     e = qnt::launch_gemv4_one(d, codes, meta, z0, X, Y, xbf16, st, s, &handled);
+    if (handled || e != cudaSuccess) return e;
+  }
+  if (!force_simt && M >= 2 && M <= 4) {
+    e = qnt::launch_gemv1_multi(d, codes, meta, X, Y, M, xbf16, st, s, &handled);
     if (handled || e != cudaSuccess) return e;
   }
   if (!force_simt && M >= 3) {

@@ -8,8 +8,8 @@ metadata must match bit-exactly) and the oracle's binary64 GEMV/GEMM on those
 rows checks the library's outputs element by element.
 
 Shapes: the Llama-7B decode GEMVs (INT4 g128, batch 1), the FP4 / AFPQ / RaZeR
-K=4096 N=14336 case (batch 1 and 4), the Llama-70B small-batch GEMMs (INT4
-g128, bf16 activations, M = 1..128) and the selective-precision stack (INT8
+K=4096 N=14336 case (batch 1, 2 and 4), the Llama-70B small-batch GEMMs (INT4
+g128, bf16 activations, M = 1..4 and 8..128) and the selective-precision stack (INT8
 per-channel down_proj, FP16 lm_head; batch 1 and 16)."""
 import numpy as np
 import pytest
@@ -56,12 +56,15 @@ def test_llama7b_decode_int4_g128(N, K):
 
 @pytest.mark.parametrize("fmt", [orc.FP4, orc.AFPQ, orc.RAZER])
 def test_fp4_family_k4096_n14336(fmt):
-    _check(fmt, 14336, 4096, 128, [1, 4], 0, seed=31 + fmt)
+    _check(fmt, 14336, 4096, 128, [1, 2, 4], 0, seed=31 + fmt)
 
 
 @pytest.mark.parametrize("N,K", [(10240, 8192), (28672, 8192), (8192, 28672)])
 def test_llama70b_small_batch_int4(N, K):
-    _check(orc.INT4, N, K, 128, [1, 8, 16, 32, 64, 128], 1, seed=N ^ K)
+    # M = 2..4 take the batch-1 kernel with the vectors sharing its MMAs (at
+    # K = 8192, N = 28672 with one ring slot per warp), or the tcgen05 GEMM
+    # where four activation images do not fit (K = 28672, M = 3, 4)
+    _check(orc.INT4, N, K, 128, [1, 2, 3, 4, 8, 16, 32, 64, 128], 1, seed=N ^ K)
 
 
 def test_selective_precision_stack_modules():

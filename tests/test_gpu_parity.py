@@ -154,11 +154,13 @@ def test_gemm_rows_equal_gemv():
 
 
 @pytest.mark.parametrize("fmt,M", [(orc.INT8, 1), (orc.FP16, 1), (orc.INT8, 3), (orc.INT4, 1), (orc.INT4, 2),
-                                   (orc.INT4, 16), (orc.RAZER, 2)])
+                                   (orc.INT4, 16), (orc.RAZER, 2), (orc.FP4, 4), (orc.AFPQ, 2)])
 def test_largest_k_every_path(fmt, M):
-    """K = QNT_MAX_GEMV_K on every kernel a call can take (the batch-1 kernel,
-    the CUDA-core kernel at batch 1-3, the tcgen05 GEMM): the activation
-    vector fits in shared memory next to each kernel's weight ring."""
+    """K = QNT_MAX_GEMV_K on every kernel a call can take (the batch-1 kernel
+    with one vector and with two sharing its MMAs, the CUDA-core kernel, the
+    tcgen05 GEMM, which takes four vectors here since four images do not fit
+    next to a ring): the activations fit in shared memory next to each
+    kernel's weight ring."""
     Q = H.q()
     N, K, g = 72, Q.QNT_MAX_GEMV_K, 128
     ref, pc, pm = _oracle_packed(fmt, N, K, g, seed=K + fmt + M)

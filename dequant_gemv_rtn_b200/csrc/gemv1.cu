@@ -541,8 +541,10 @@ gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
       }
       const uint32_t ca = sbase + (uint32_t)L.ring + (uint32_t)slot * (uint32_t)kB1SlotBytes + coff;
       float yacc = 0.0f;
-      if (MV > 1 || (nb == RB && G == 128 && FMT != QNT_FP4_AFPQ && (GK & 1) == 0)) {
-       if constexpr (MV == 1) {
+      // AFPQ's full items at g = 128 take the vector-general path below at any MV
+      constexpr bool kGeneral = MV > 1 || (FMT == QNT_FP4_AFPQ && G == 128);
+      if (MV > 1 || (nb == RB && G == 128 && (FMT == QNT_FP4_AFPQ || (GK & 1) == 0))) {
+       if constexpr (!kGeneral) {
         // ---- full item, g = 128, an even number of groups per row: the lane's
         // epilogue blocks are ei * NQ + q, q < NQ (two consecutive groups of its
         // row, the first of even index, so both scales are one aligned 32-bit
@@ -592,20 +594,23 @@ gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
           yacc += ea[q] * v - eb[q];
         }
        } else {
-        // ---- several vectors (g = 128, full items, not AFPQ: the launcher's
-        // conditions).  Set q holds blocks q + NQ i (i < S); the lane's epilogue
-        // blocks are NQ ei + q, q < NQ: NQ consecutive groups of its row whose
-        // scales (and INT4 zero points) are one aligned load, as the group index
-        // of the first is a multiple of NQ (K is a multiple of 1024).
-        static_assert(G == 128 && FMT != QNT_FP4_AFPQ, "several vectors: g = 128, not AFPQ");
+        // ---- several vectors (g = 128, full items: the launcher's conditions),
+        // or AFPQ's full items at g = 128.
+        // Set q holds blocks q + NQ i (i < S); the lane's epilogue blocks are
+        // NQ ei + q, q < NQ: NQ consecutive groups of its row whose scales (and
+        // INT4 zero points) are aligned loads, as the group index of the first
+        // is a multiple of NQ (K is a multiple of 1024).
+        static_assert(G == 128, "several vectors: g = 128");
         const uint32_t fe = fr0 + (uint32_t)(NQ * ei);
-        uint32_t sw[NQ / 2];                                   // the NQ fp16 scales, two per word
-        if constexpr (NQ == 8) {
-          const uint4 t = lds128a(M.ms_a + 2u * fe);
-          sw[0] = t.x; sw[1] = t.y; sw[2] = t.z; sw[3] = t.w;
-        } else {
-          const uint2 t = lds64a(M.ms_a + 2u * fe);
-          sw[0] = t.x; sw[1] = t.y;
+        uint32_t sw[NQ / 2] = {};                              // the NQ fp16 scales, two per word (AFPQ: per set)
+        if constexpr (FMT != QNT_FP4_AFPQ) {
+          if constexpr (NQ == 8) {
+            const uint4 t = lds128a(M.ms_a + 2u * fe);
+            sw[0] = t.x; sw[1] = t.y; sw[2] = t.z; sw[3] = t.w;
+          } else {
+            const uint2 t = lds64a(M.ms_a + 2u * fe);
+            sw[0] = t.x; sw[1] = t.y;
+          }
         }
         uint32_t zw = 0u;                                      // INT4: the NQ zero points, a nibble each
         if (FMT == QNT_INT4_ASYM) zw = NQ == 8 ? lds32a(M.mz_a + (fe >> 1)) : lds16a(M.mz_a + (fe >> 1));
@@ -633,14 +638,19 @@ gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
           for (int jj = 0; jj < 4; ++jj)
 #pragma unroll
             for (int i = 0; i < S; ++i) word_mma<FMT>((&cv[i].x)[jj], jj, bx, d[i], dn[i], sv16[i]);
-          float v = d[0][0] + d[0][3];
+          float v = d[0][0] + d[0][3], vn = dn[0][0] + dn[0][3];
 #pragma unroll
           for (int i = 1; i < S; ++i)
-            if (ei == i) v = d[i][0] + d[i][3];
+            if (ei == i) { v = d[i][0] + d[i][3]; vn = dn[i][0] + dn[i][3]; }
           const float2 sc = lds64fa(xsv + 8u * q);             // (c / 2^e, group sum of x) of vector ve
-          const float sq = h2f((sw[q >> 1] >> (16 * (q & 1))) & 0xFFFFu);
-          const float zq = FMT == QNT_INT4_ASYM ? (float)((zw >> (4 * q)) & 15u) : 0.0f;
-          yacc += sq * (sc.x * v - zq * sc.y);
+          if (FMT == QNT_FP4_AFPQ) {                             // positive part times s+, negative times s-
+            const uint32_t w2 = lds32a(M.ms_a + 4u * (fe + (uint32_t)q));
+            yacc += sc.x * (h2f(w2 & 0xFFFFu) * v + h2f(w2 >> 16) * vn);
+          } else {
+            const float sq = h2f((sw[q >> 1] >> (16 * (q & 1))) & 0xFFFFu);
+            const float zq = FMT == QNT_INT4_ASYM ? (float)((zw >> (4 * q)) & 15u) : 0.0f;
+            yacc += sq * (sc.x * v - zq * sc.y);
+          }
         }
         if (!rowok) yacc = 0.0f;
        }
@@ -937,8 +947,9 @@ cudaError_t launch_gemv1_multi(const qnt_desc& d, const void* codes, const void*
   switch (d.fmt) {
     case QNT_INT4_ASYM: QNT_B1M(QNT_INT4_ASYM)
     case QNT_FP4_E2M1: QNT_B1M(QNT_FP4_E2M1)
+    case QNT_FP4_AFPQ: QNT_B1M(QNT_FP4_AFPQ)
     case QNT_FP4_RAZER: QNT_B1M(QNT_FP4_RAZER)
-    default: return cudaSuccess;   // AFPQ: not handled here
+    default: return cudaSuccess;
   }
 #undef QNT_B1M
 }

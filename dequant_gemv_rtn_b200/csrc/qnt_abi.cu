@@ -47,7 +47,7 @@ int check(const qnt_desc* d) {
 
 // Y[m] = W x[m], m < M.  Kernel choice (measured on B200 with L2-cold weights):
 //   one vector, 4-bit formats       -> batch-1 kernel (mma.sync tensor cores)
-//   2..4 vectors, INT4 / FP4 / RaZeR, group 128, K a multiple of 1024
+//   2..4 vectors, 4-bit formats, group 128, K a multiple of 1024
 //                                   -> the batch-1 kernel, the vectors sharing its MMAs
 //   3..128 vectors, 4-bit formats   -> tcgen05 GEMM, one pass over the weights
 //   2 vectors otherwise, INT8, FP16 -> CUDA-core multi-vector kernel (passes of 8)

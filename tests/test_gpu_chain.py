@@ -172,6 +172,42 @@ def test_gemv_seq_independent_steps_and_tiny_shapes():
         _check_chain(mats, xs, ys, xdt, f"independent rep {rep}")
 
 
+@pytest.mark.parametrize("fmt,g", [(orc.INT4, 128), (orc.AFPQ, 128), (orc.RAZER, 64), (orc.FP4, 32)])
+def test_gemv_seq_shared_x_and_waits_back(fmt, g):
+    """Steps that read the same x with no new dependency keep one activation
+    image (the second and third step on x0, the fifth after the fourth), one of
+    them with rows on few CTAs (N = 40); steps that wait several steps back
+    (step 3 for step 0, step 4 for step 0 as well, step 6 for step 4); a step
+    with a larger K than the others in between (8192).  Two calls in a row;
+    every y poisoned with NaN before each."""
+    Q = H.q()
+    xdt = 0
+    #            (N, K),       x source,        wait
+    plan = [((1200, 2048), "x0", 0), ((40, 2048), "x0", 0), ((1000, 2048), "x0", 0),
+            ((2048, 1024), ("y", 0), 3), ((512, 1024), ("y", 0), 4), ((256, 8192), "xb", 0),
+            ((300, 512), ("y", 4), 2)]
+    mats = [_packed(fmt, N, K, g, 700 + i) for i, ((N, K), _, _) in enumerate(plan)]
+    x0 = H.x_tensor(H.to_x_bits(synth.activations(1, 2048, seed=70), xdt))
+    xb = H.x_tensor(H.to_x_bits(synth.activations(1, 8192, seed=71), xdt))
+    ys = [torch.full((N,), NAN16, dtype=torch.int16, device="cuda") for (N, _), _, _ in plan]
+    xs = []
+    for (N, K), src, _ in plan:
+        xs.append(x0 if src == "x0" else xb if src == "xb" else ys[src[1]][:K])
+        assert xs[-1].numel() == K
+    items = [(Q.desc(fmt, N, K, g), pc, pm, x, y, w)
+             for ((ref, pc, pm), x, y, ((N, K), _, w)) in zip(mats, xs, ys, plan)]
+    steps = Q.seq_steps(items)
+    work = H.dev_bytes(Q.qnt_gemv_seq_work_bytes(len(items)))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for rep in range(2):
+        for y in ys:
+            y.fill_(NAN16)
+        Q.qnt_gemv_seq(steps, xdt, work, st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        _check_chain(mats, xs, ys, xdt, f"continuing steps fmt={fmt} g={g} rep {rep}")
+
+
 def test_gemv_seq_llama_layers_in_cuda_graph():
     """Two Llama-7B decode layers (qkv 12288x4096, o 4096^2, gate / up 11008x4096,
     down 4096x11008; INT4 g128) as one sequence: o reads the first 4096 outputs

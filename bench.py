@@ -553,7 +553,7 @@ def run_extra_configs(args):
     for fmt, fname in ((2, "fp4"), (3, "afpq"), (4, "razer")):
         N, K = 14336, 4096
         copies = [_quantized(Q, torch, synth, fmt, N, K, GROUP, 40 + i, st) for i in range(ncopies(algo_bytes(fmt, N, K, 1)))]
-        for M in (1, 2, 4):
+        for M in (1, 2, 4, 8):
             out[f"{fname}_g128_{K}x{N}_b{M}"] = timed(fname, fmt, N, K, M, 0, copies)
         del copies
         torch.cuda.empty_cache()

@@ -327,12 +327,60 @@ __device__ __forceinline__ void word_mma(uint32_t w, int j, const uint32_t (&bx)
   }
 }
 
+// word_mma for two B operands (eight vectors: vectors 0-3 in bxa, 4-7 in bxb):
+// the word is decoded once and feeds both MMAs.
+template <int FMT>
+__device__ __forceinline__ void word_mma2(uint32_t w, int j, const uint32_t (&bxa)[8], const uint32_t (&bxb)[8],
+                                          float (&da)[4], float (&dna)[4], float (&db)[4], float (&dnb)[4],
+                                          uint32_t sv16) {
+  uint32_t h[4];
+  if (FMT == QNT_INT4_ASYM) {
+    const uint32_t w8 = w >> 8;
+    h[0] = w & 0x000F000Fu; h[1] = w8 & 0x000F000Fu; h[2] = w & 0x00F000F0u; h[3] = w8 & 0x00F000F0u;
+  } else {
+    cvt_e2m1x8(w, h[0], h[1], h[2], h[3]);
+    if (FMT == QNT_FP4_RAZER) {   // as in word_mma
+      const uint32_t tt = (w & 0x77777777u) + 0x77777777u;
+      const uint32_t spec = lop3<0x20>(w, tt, 0x88888888u);
+      uint32_t ind[4];
+      cvt_e2m1x8(spec >> 3, ind[0], ind[1], ind[2], ind[3]);
+#pragma unroll
+      for (int pp = 0; pp < 4; ++pp) h[pp] = hfma2(ind[pp], sv16, h[pp]);
+    }
+  }
+  if (FMT == QNT_FP4_AFPQ) {
+    uint32_t hp[4], hn[4];
+#pragma unroll
+    for (int pp = 0; pp < 4; ++pp) { hp[pp] = hmax2(h[pp], 0u); hn[pp] = hsub2(h[pp], hp[pp]); }
+    if (j == 0) {
+      mma_16816_z(da, hp[0], hp[1], hp[2], hp[3], bxa[0], bxa[1]);
+      mma_16816_z(dna, hn[0], hn[1], hn[2], hn[3], bxa[0], bxa[1]);
+      mma_16816_z(db, hp[0], hp[1], hp[2], hp[3], bxb[0], bxb[1]);
+      mma_16816_z(dnb, hn[0], hn[1], hn[2], hn[3], bxb[0], bxb[1]);
+    } else {
+      mma_16816(da, hp[0], hp[1], hp[2], hp[3], bxa[2 * j], bxa[2 * j + 1]);
+      mma_16816(dna, hn[0], hn[1], hn[2], hn[3], bxa[2 * j], bxa[2 * j + 1]);
+      mma_16816(db, hp[0], hp[1], hp[2], hp[3], bxb[2 * j], bxb[2 * j + 1]);
+      mma_16816(dnb, hn[0], hn[1], hn[2], hn[3], bxb[2 * j], bxb[2 * j + 1]);
+    }
+  } else {
+    if (j == 0) {
+      mma_16816_z(da, h[0], h[1], h[2], h[3], bxa[0], bxa[1]);
+      mma_16816_z(db, h[0], h[1], h[2], h[3], bxb[0], bxb[1]);
+    } else {
+      mma_16816(da, h[0], h[1], h[2], h[3], bxa[2 * j], bxa[2 * j + 1]);
+      mma_16816(db, h[0], h[1], h[2], h[3], bxb[2 * j], bxb[2 * j + 1]);
+    }
+  }
+}
+
 // ------------------------------------------------------------------ kernel
 template <int FMT, int G, int MAXS, int MV>
 __global__ void __launch_bounds__(kB1Threads, 1)
 gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
   constexpr int GPB = 128 / G;        // groups per block
-  constexpr int S = 4 / (GPB * MV);   // blocks per set (accumulators)
+  constexpr int MVc = MV > 4 ? 4 : MV;   // vectors per B operand (eight vectors: two B operands)
+  constexpr int S = 4 / (GPB * MVc);  // blocks per set (accumulators)
   constexpr int NQ = kB1Blocks / S;   // sets per full item
   constexpr int RB = kB1Blocks;
   constexpr int C = kB1Warps;
@@ -456,11 +504,11 @@ gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
   const int g = lane >> 2, r = lane & 3;
   const int hp = lane >> 3;                                    // B column pair of this lane
   const bool bload = (r * GPB) / 4 == hp % GPB;                // this lane's chunk lies in the pair's group
-  const int bsel = hp / (GPB * MV);                            // block of the set that feeds the pair
-  const int ei = r / (GPB * MV), eh = r % GPB;                 // epilogue: accumulator, group in block
+  const int bsel = hp / (GPB * MVc);                           // block of the set that feeds the pair
+  const int ei = r / (GPB * MVc), eh = r % GPB;                // epilogue: accumulator, group in block
   // several vectors (MV > 1, g = 128): column pair hp carries vector hp % MV of
   // block hp / MV of the set, and lane 4g + r's result belongs to vector r % MV
-  const int vb = hp % MV, ve = r % MV;
+  const int vb = hp % MVc, ve = r % MVc;
   const int IMGV = 2 * P.kmax, XSV = (P.kmax / 128) * GPB * 8;   // bytes per vector: image, factor table
   const uint32_t coff = 64u * g + 16u * (uint32_t)(r ^ ((g >> 1) & 3));
   const uint32_t xoff = 16u * (uint32_t)(4 * ((lane >> 2) & 1) + r);
@@ -540,7 +588,7 @@ gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
         break;
       }
       const uint32_t ca = sbase + (uint32_t)L.ring + (uint32_t)slot * (uint32_t)kB1SlotBytes + coff;
-      float yacc = 0.0f;
+      float yacc = 0.0f, yacc2 = 0.0f;   // yacc2: eight vectors, the lane's second one (r + 4)
       // AFPQ's full items at g = 128 take the vector-general path below at any MV
       constexpr bool kGeneral = MV > 1 || (FMT == QNT_FP4_AFPQ && G == 128);
       if (MV > 1 || (nb == RB && G == 128 && (FMT == QNT_FP4_AFPQ || (GK & 1) == 0))) {
@@ -593,6 +641,47 @@ gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
             if (ei == i) v = d[i][0] + d[i][3];
           yacc += ea[q] * v - eb[q];
         }
+       } else if constexpr (MV == 8) {
+        // ---- eight vectors (g = 128, full items): two B operands, vectors 0-3
+        // and 4-7, column pair hp carries vectors hp and hp + 4 of block q of set
+        // q (one block per set), every code word is decoded once for both MMAs,
+        // and lane 4g + r ends with vectors r and r + 4 of its row.
+        const uint32_t fe = fr0;                               // the item's 8 groups of the row
+        const uint32_t xs0 = xs2_a + (uint32_t)(r * XSV) + 8u * (uint32_t)b0;
+        const uint32_t xs1 = xs2_a + (uint32_t)((r + 4) * XSV) + 8u * (uint32_t)b0;
+        const uint32_t xa0 = ximg_a + (uint32_t)(hp * IMGV) + 256u * (uint32_t)b0 + xoff;
+        const uint32_t xa1 = ximg_a + (uint32_t)((hp + 4) * IMGV) + 256u * (uint32_t)b0 + xoff;
+#pragma unroll 2
+        for (int q = 0; q < 8; ++q) {
+          const uint4 cv = lds128a(ca + 512u * (uint32_t)q);
+          const uint4 a0 = lds128a(xa0 + 256u * q), a1 = lds128a(xa0 + 256u * q + 128u);
+          const uint4 c0 = lds128a(xa1 + 256u * q), c1 = lds128a(xa1 + 256u * q + 128u);
+          const uint32_t bxa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+          const uint32_t bxb[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          uint32_t sv16 = 0u;
+          if (FMT == QNT_FP4_RAZER) {
+            const uint32_t sel = meta_sel2(M, fr0 + (uint32_t)q);
+            const uint32_t sv2 = ((sel & 2u) ? 0x4C00u : 0x4900u) | ((sel & 1u) ? 0x8000u : 0u);   // 2 sv: +-16 or +-10
+            sv16 = sv2 | (sv2 << 16);
+          }
+          float da[4], dna[4], db[4], dnb[4];
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) word_mma2<FMT>((&cv.x)[jj], jj, bxa, bxb, da, dna, db, dnb, sv16);
+          const float v0 = da[0] + da[3], v1 = db[0] + db[3];
+          const float2 sc0 = lds64fa(xs0 + 8u * q), sc1 = lds64fa(xs1 + 8u * q);
+          if (FMT == QNT_FP4_AFPQ) {
+            const uint32_t w2 = lds32a(M.ms_a + 4u * (fe + (uint32_t)q));
+            const float sp = h2f(w2 & 0xFFFFu), sn = h2f(w2 >> 16);
+            yacc += sc0.x * (sp * v0 + sn * (dna[0] + dna[3]));
+            yacc2 += sc1.x * (sp * v1 + sn * (dnb[0] + dnb[3]));
+          } else {
+            const float sq = meta_scale(M, fe + (uint32_t)q);
+            const float zq = FMT == QNT_INT4_ASYM ? (float)meta_zero4(M, fe + (uint32_t)q) : 0.0f;
+            yacc += sq * (sc0.x * v0 - zq * sc0.y);
+            yacc2 += sq * (sc1.x * v1 - zq * sc1.y);
+          }
+        }
+        if (!rowok) yacc = yacc2 = 0.0f;
        } else {
         // ---- several vectors (g = 128, full items: the launcher's conditions),
         // or AFPQ's full items at g = 128.
@@ -723,6 +812,11 @@ gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
         yacc += __shfl_xor_sync(0xffffffffu, yacc, 1);
         yacc += __shfl_xor_sync(0xffffffffu, yacc, 2);
         if (r == 0 && rowok) part[rl * KBR + br] = yacc;
+      } else if constexpr (MV == 8) {   // lane r ends with vectors r and r + 4
+        if (rowok) {
+          part[r * P.part_cap + rl * KBR + br] = yacc;
+          part[(r + 4) * P.part_cap + rl * KBR + br] = yacc2;
+        }
       } else {   // lanes r and r ^ 2 hold the same vector when MV = 2; lane r < MV ends with vector r
         if (MV == 2) yacc += __shfl_xor_sync(0xffffffffu, yacc, 2);
         if (r < MV && rowok) part[r * P.part_cap + rl * KBR + br] = yacc;
@@ -933,7 +1027,7 @@ cudaError_t launch_gemv4_one(const qnt_desc& d, const void* codes, const void* m
 cudaError_t launch_gemv1_multi(const qnt_desc& d, const void* codes, const void* meta, const void* X, void* Y, int M,
                               int xbf16, int* st, cudaStream_t s, bool* handled) {
   *handled = false;
-  if (M < 2 || M > 4 || d.group != 128 || d.K % 1024 != 0) return cudaSuccess;
+  if (M < 2 || M > 8 || d.group != 128 || d.K % 1024 != 0) return cudaSuccess;
   qnt_seq_step one = {};
   one.desc = d;
   one.codes = codes;
@@ -942,8 +1036,9 @@ cudaError_t launch_gemv1_multi(const qnt_desc& d, const void* codes, const void*
   one.y = Y;
   one.wait = 0;
 #define QNT_B1M(FMT)                                                                                       \
-  return M == 2 ? b1_launch<FMT, 128, 1, 2>(&one, 1, xbf16, nullptr, st, s, false, handled, M)            \
-                : b1_launch<FMT, 128, 1, 4>(&one, 1, xbf16, nullptr, st, s, false, handled, M);
+  return M == 2   ? b1_launch<FMT, 128, 1, 2>(&one, 1, xbf16, nullptr, st, s, false, handled, M)          \
+         : M <= 4 ? b1_launch<FMT, 128, 1, 4>(&one, 1, xbf16, nullptr, st, s, false, handled, M)          \
+                  : b1_launch<FMT, 128, 1, 8>(&one, 1, xbf16, nullptr, st, s, false, handled, M);
   switch (d.fmt) {
     case QNT_INT4_ASYM: QNT_B1M(QNT_INT4_ASYM)
     case QNT_FP4_E2M1: QNT_B1M(QNT_FP4_E2M1)

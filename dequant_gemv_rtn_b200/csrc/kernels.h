@@ -29,7 +29,7 @@ cudaError_t launch_gemv_simt(const qnt_desc& d, const void* codes, const void* m
 cudaError_t launch_gemv4_one(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
                              int xbf16, int* st, cudaStream_t s, bool* handled);
 
-// Two to four vectors of the 4-bit formats, group 128, K a multiple of 1024:
+// Two to eight vectors of the 4-bit formats, group 128, K a multiple of 1024:
 // the batch-1 kernel with the vectors sharing every MMA (gemv1.cu).
 // *handled = false when the case is not covered or does not fit.
 cudaError_t launch_gemv1_multi(const qnt_desc& d, const void* codes, const void* meta, const void* X, void* Y, int M,

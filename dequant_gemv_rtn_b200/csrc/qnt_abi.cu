@@ -47,7 +47,7 @@ int check(const qnt_desc* d) {
 
 // Y[m] = W x[m], m < M.  Kernel choice (measured on B200 with L2-cold weights):
 //   one vector, 4-bit formats       -> batch-1 kernel (mma.sync tensor cores)
-//   2..4 vectors, 4-bit formats, group 128, K a multiple of 1024
+//   2..8 vectors, 4-bit formats, group 128, K a multiple of 1024
 //                                   -> the batch-1 kernel, the vectors sharing its MMAs
 //   3..128 vectors, 4-bit formats   -> tcgen05 GEMM, one pass over the weights
 //   2 vectors otherwise, INT8, FP16 -> CUDA-core multi-vector kernel (passes of 8)
@@ -66,7 +66,7 @@ cudaError_t dispatch_gemm(const qnt_desc& d, const void* codes, const void* meta
     e = qnt::launch_gemv4_one(d, codes, meta, z0, X, Y, xbf16, st, s, &handled);
     if (handled || e != cudaSuccess) return e;
   }
-  if (!force_simt && M >= 2 && M <= 4) {
+  if (!force_simt && M >= 2 && M <= 8) {
     e = qnt::launch_gemv1_multi(d, codes, meta, X, Y, M, xbf16, st, s, &handled);
     if (handled || e != cudaSuccess) return e;
   }

@@ -203,7 +203,7 @@ int qnt_gemv(const qnt_desc* desc, const void* d_codes, const void* d_meta,
  *   d_Y        device, [M][N] in the same type, written.
  * Same ordering rule (the immediately preceding kernel on the stream must not
  * write d_codes or d_meta) and accuracy statement as qnt_gemv.  Batches of 2 to
- * 4 rows of the 4-bit formats with group 128 and K a multiple of 1024 run on
+ * 8 rows of the 4-bit formats with group 128 and K a multiple of 1024 run on
  * the batch-1 kernel, the rows sharing its tensor-core MMAs, when their
  * activations fit in shared memory next to its weight ring; the other batches
  * of 3 to 128 rows of the 4-bit formats run on the tcgen05 tensor cores in one

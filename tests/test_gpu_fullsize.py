@@ -8,7 +8,7 @@ metadata must match bit-exactly) and the oracle's binary64 GEMV/GEMM on those
 rows checks the library's outputs element by element.
 
 Shapes: the Llama-7B decode GEMVs (INT4 g128, batch 1), the FP4 / AFPQ / RaZeR
-K=4096 N=14336 case (batch 1, 2 and 4), the Llama-70B small-batch GEMMs (INT4
+K=4096 N=14336 case (batch 1, 2, 4 and 8), the Llama-70B small-batch GEMMs (INT4
 g128, bf16 activations, M = 1..4 and 8..128) and the selective-precision stack (INT8
 per-channel down_proj, FP16 lm_head; batch 1 and 16)."""
 import numpy as np
@@ -56,7 +56,7 @@ def test_llama7b_decode_int4_g128(N, K):
 
 @pytest.mark.parametrize("fmt", [orc.FP4, orc.AFPQ, orc.RAZER])
 def test_fp4_family_k4096_n14336(fmt):
-    _check(fmt, 14336, 4096, 128, [1, 2, 4], 0, seed=31 + fmt)
+    _check(fmt, 14336, 4096, 128, [1, 2, 4, 8], 0, seed=31 + fmt)
 
 
 @pytest.mark.parametrize("N,K", [(10240, 8192), (28672, 8192), (8192, 28672)])

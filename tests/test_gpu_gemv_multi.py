@@ -1,11 +1,12 @@
-"""GPU parity of qnt_gemm with 2 to 4 activation vectors on the batch-1 tensor-core
+"""GPU parity of qnt_gemm with 2 to 8 activation vectors on the batch-1 tensor-core
 kernel (the 4-bit formats, group 128, K a multiple of 1024: the vectors share
-every mma.sync, each in its own B column pair) against the CPU oracle.
+every mma.sync, each in its own B column pair; eight vectors use two B operands
+per decoded word) against the CPU oracle.
 
 Shapes: one 128-row tile's worth of row groups on 25 CTAs with a ragged count of
 rows (200); 1000 rows at K = 4096 (four runs of K per row); 513 row groups, more
-than there are SMs, so CTAs hold 3 or 4 row groups.  M = 3 leaves the fourth
-vector slot empty (an image of zeros that nothing reads back).  The cases the
+than there are SMs, so CTAs hold 3 or 4 row groups.  M = 3 and M = 5 leave
+vector slots empty (images of zeros that nothing reads back).  The cases the
 launcher does not take (group 32 or 64, K not a multiple of 1024) go to the other
 kernels and are checked here too, so every M in 2..4 is covered whatever the
 dispatch.  Tolerance: 4e-3 * sum_k |dq x| per element, as for every GEMV."""
@@ -29,7 +30,7 @@ def _packed(fmt, N, K, g, seed):
 
 @pytest.mark.parametrize("fmt", [orc.INT4, orc.FP4, orc.AFPQ, orc.RAZER])
 @pytest.mark.parametrize("N,K", [(200, 2048), (1000, 4096), (4104, 1024)])
-@pytest.mark.parametrize("M", [2, 3, 4])
+@pytest.mark.parametrize("M", [2, 3, 4, 5, 8])
 def test_gemv_multi_parity(fmt, N, K, M):
     ref, pc, pm = _packed(fmt, N, K, 128, seed=7 * N + K + M + fmt)
     for xdt in (0, 1):
@@ -41,7 +42,7 @@ def test_gemv_multi_parity(fmt, N, K, M):
 
 @pytest.mark.parametrize("fmt,g,K", [(orc.AFPQ, 64, 2048), (orc.INT4, 64, 2048), (orc.RAZER, 128, 2304),
                                      (orc.FP4, 32, 1024), (orc.INT4, 32, 3072)])
-@pytest.mark.parametrize("M", [2, 3, 4])
+@pytest.mark.parametrize("M", [2, 4, 8])
 def test_gemv_multi_cases_taken_elsewhere(fmt, g, K, M):
     N = 264
     ref, pc, pm = _packed(fmt, N, K, g, seed=K + g + M)
@@ -51,7 +52,7 @@ def test_gemv_multi_cases_taken_elsewhere(fmt, g, K, M):
     H.assert_within_tol(y, yref, aref, f"M={M} fmt={fmt} g{g} K={K}", 0)
 
 
-@pytest.mark.parametrize("M", [2, 4])
+@pytest.mark.parametrize("M", [2, 4, 8])
 def test_gemv_multi_vectors_are_independent(M):
     """Each vector meets only its own B column pair, so a batch of copies of
     one vector gives that vector's outputs in every row, bit for bit, and a

@@ -830,7 +830,8 @@ cudaError_t gt_launch(const qnt_desc& d, const void* codes, const void* meta, lo
 
 }  // namespace
 
-// 1..128 activation rows (dispatched for 3..128), 4-bit formats, one pass over the weights.
+// 1..128 activation rows (dispatched for 9..128, and for 3..8 where the batch-1 kernel's
+// activation images do not fit), 4-bit formats, one pass over the weights.
 cudaError_t launch_gemm_tc(const qnt_desc& d, const void* codes, const void* meta, long z0, const void* X, void* Y,
                            int M, int xbf16, int* st, cudaStream_t s, bool* handled) {
   *handled = false;

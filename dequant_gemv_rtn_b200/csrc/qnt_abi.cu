@@ -49,7 +49,7 @@ int check(const qnt_desc* d) {
 //   one vector, 4-bit formats       -> batch-1 kernel (mma.sync tensor cores)
 //   2..8 vectors, 4-bit formats, group 128, K a multiple of 1024
 //                                   -> the batch-1 kernel, the vectors sharing its MMAs
-//   3..128 vectors, 4-bit formats   -> tcgen05 GEMM, one pass over the weights
+//   3..128 vectors otherwise        -> tcgen05 GEMM, one pass over the weights
 //   2 vectors otherwise, INT8, FP16 -> CUDA-core multi-vector kernel (passes of 8)
 // QNT_FORCE_SIMT=1 selects the CUDA-core multi-vector kernel everywhere (used to
 // test every path on the same inputs).

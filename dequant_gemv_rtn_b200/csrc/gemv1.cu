@@ -1,6 +1,7 @@
 // gemv1.cu -- batch-1 fused-dequant GEMV for the 4-bit formats on the tensor
-// cores (mma.sync), launched once per GEMV (qnt_gemv) or once for a whole
-// sequence of GEMVs (qnt_gemv_seq, a persistent kernel).
+// cores (mma.sync), launched once per GEMV (qnt_gemv), once for a whole
+// sequence of GEMVs (qnt_gemv_seq, a persistent kernel), or once for 2 to 8
+// activation vectors (qnt_gemm).
 //
 // What it computes is the decode-time GEMV of the RTN page ("Is (Selective)
 // Round-To-Nearest Quantization All You Need?", English abstract: token
@@ -31,11 +32,12 @@
 //    (block, group) pair: the scale / zero-point epilogue runs once per set in
 //    all 32 lanes.  The products that pair one block's weights with another
 //    block's activations land in accumulator entries that are never read.
-//  * Activations: the bulk copy of x lands in shared memory; the consumers
-//    rewrite it in place as the B-operand image (each block scaled by an exact
-//    power of two that puts its maximum in [2^14, 2^15), undone in fp32 by the
-//    epilogue) with, per (block, group), the scale factor and the group sum of
-//    x (INT4 zero point: -s z sum x).
+//  * Activations: each warp reads its blocks of x from global memory (at L2:
+//    in a sequence another SM may have just written x) and writes them as the
+//    B-operand image (each block scaled by an exact power of two that puts its
+//    maximum in [2^14, 2^15), undone in fp32 by the epilogue) with, per
+//    (block, group), the scale factor and the group sum of x (INT4 zero point:
+//    -s z sum x).
 //  * Sequence: each step may wait for every earlier step of the launch (its x is
 //    then an earlier step's y): one thread polls the per-step completion
 //    counters in the caller's workspace (acquire), and each CTA bumps the counter
@@ -44,6 +46,11 @@
 //  * qnt_gemv: the same kernel with one step and programmatic dependent launch;
 //    the weights are requested before griddepcontrol.wait, the activations
 //    after it.
+//  * qnt_gemm with 2 to 8 vectors (template parameter MV = 2, 4, 8; g = 128, K a
+//    multiple of 1024): the B column pairs that batch 1 spends on several blocks
+//    of one vector carry the vectors instead (MV = 8: two B operands per decoded
+//    word), each vector with its own image, factor table and partial sums, so
+//    the decode and the codes traffic per weight stay those of batch 1.
 // Every wait is bounded by the global timer; on expiry the kernel reports
 // QNT_ERR_TIMEOUT, stops issuing work, drains its copies and returns.
 #include <cstring>

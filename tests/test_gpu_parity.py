@@ -67,6 +67,39 @@ def test_quantize_edge_groups():
         H.assert_quant_equal(got, orc.quantize(fmt, W, g), f"edge fmt={fmt}")
 
 
+@pytest.mark.parametrize("fmt", [orc.INT4, orc.INT8])
+def test_quantize_ties_and_near_ties(fmt):
+    """Integer codes round the quotient w / S to nearest, ties to even.  Groups
+    whose scale is exact (S = 1, 1/16) or not (S = fp16(0.1), from a range of
+    1.5) hold weights on half-integer quotients and one binary32 ulp to either
+    side of them, so that every rounding of the quotient is decided exactly at
+    or next to a tie; codes and metadata must equal the oracle's bit for bit."""
+    K, g = 256, 128
+    rows = []
+    for span in (15.0, 15.0 / 16, 1.5):
+        if fmt == orc.INT4:   # min 0, max span: S = fp16(span / 15), z = 0
+            S = float(np.float16(span / 15))
+            ties = [(k + 0.5) * S for k in range(15)]
+        else:                 # max |w| = 127 S
+            S = float(np.float16(span / 15))
+            ties = [(k + 0.5) * S for k in range(-127, 127)]
+        t = np.array(ties, dtype=np.float32)
+        vals = np.concatenate([t, np.nextafter(t, np.float32(np.inf)), np.nextafter(t, np.float32(-np.inf))])
+        row = np.resize(vals, K).astype(np.float32)
+        for c in range(0, K, g):   # every group spans the whole range
+            if fmt == orc.INT4:
+                row[c], row[c + 1] = 0.0, np.float32(span)
+            else:
+                row[c], row[c + 1] = np.float32(127 * S), np.float32(-127 * S)
+        rows.append(row)
+    W = np.stack(rows).astype(np.float32)
+    codes, meta, st = H.gpu_quantize(fmt, torch.from_numpy(W).cuda(), g)
+    assert int(st.item()) == 0
+    gg = g if fmt in FOUR else K
+    ref = orc.quantize(fmt, W, g)
+    H.assert_quant_equal(H.unpack_rows(fmt, W.shape[0], K, gg, codes, meta), ref, f"ties fmt={fmt}")
+
+
 @pytest.mark.parametrize("fmt", ALL)
 def test_quantize_status_codes(fmt):
     K = 256

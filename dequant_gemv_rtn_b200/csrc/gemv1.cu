@@ -712,7 +712,11 @@ gemv1_kernel(const __grid_constant__ B1Params<MAXS> P) {
         if (FMT == QNT_INT4_ASYM) zw = NQ == 8 ? lds32a(M.mz_a + (fe >> 1)) : lds16a(M.mz_a + (fe >> 1));
         const uint32_t xsv = xs2_a + (uint32_t)(ve * XSV) + 8u * (uint32_t)(b0 + NQ * ei);   // vector ve's factors
         const uint32_t xa = ximg_a + (uint32_t)(vb * IMGV) + 256u * (uint32_t)(b0 + NQ * bsel) + xoff;
-#pragma unroll
+        // AFPQ with one or two vectors: both parts of a set's blocks are 32 or 16
+        // accumulators; one set at a time keeps them in registers (no spills;
+        // measured 3.5 % faster at batch 1, 1.5 % slower at batch 2)
+        constexpr int kSetUnroll = (FMT == QNT_FP4_AFPQ && MV <= 2) ? 1 : NQ;
+#pragma unroll kSetUnroll
         for (int q = 0; q < NQ; ++q) {
           uint4 cv[S];
 #pragma unroll
